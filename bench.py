@@ -1,0 +1,467 @@
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one pass of the whole hot path over one batch: copy-on-write block
+copies (when the workload forks), the cache write of each sequence's new
+token, and paged decode attention (plus its log-sum-exp merge when contexts
+are split).  Inputs are seeded and synthetic, resident in HBM when timing
+starts; the K/V of a step (1.5 GB for the default workload) is far larger
+than the 126 MB L2, so no explicit flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+
+Prints one JSON line (rank 0).  Multi-GPU runs are independent replicas, one
+process per GPU (torchrun); time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn: achieved HBM GB/s (% of B200 peak), µs/step, seqs/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="opt13b_f16")
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# workload and byte model
+# ---------------------------------------------------------------------------
+def decode_bytes(lay):
+    """Algorithmic bytes of one decode call: K+V of every context token, q
+    and out, the block-table entries read and the context lengths."""
+    from paged_kv_cache_480_b200.workloads import DTYPE_BYTES
+    dt = DTYPE_BYTES[lay.dtype]
+    lens = lay.context_lens.astype(np.int64)
+    kv = int(lens.sum()) * lay.num_kv_heads * lay.head_size * dt * 2
+    qo = 2 * lay.num_seqs * lay.num_heads * lay.head_size * dt
+    tables = int((-(-lens // lay.block_size)).sum()) * 4
+    return kv + qo + tables + 4 * lay.num_seqs
+
+
+def cache_write_bytes(lay):
+    """reshape_and_cache of one token per sequence: read k, v; write them; read slots."""
+    from paged_kv_cache_480_b200.workloads import DTYPE_BYTES
+    row = lay.num_kv_heads * lay.head_size * DTYPE_BYTES[lay.dtype]
+    return lay.num_seqs * (4 * row + 8)
+
+
+def build_workload(name, block_size, device):
+    from paged_kv_cache_480_b200 import workloads as wl
+    if name == "cow_bf16":
+        return build_cow_state(device)
+    lay = wl.make_layout(name, block_size=block_size)
+    ten = wl.make_tensors(lay, device=device)
+    return lay, ten, None
+
+
+def build_cow_state(device):
+    """The parallel-sampling workload at its first generation step: prompts
+    prefilled and forked, so the step's first own token of every writing
+    sample triggers copy-on-write of the shared partial block."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    from paged_kv_cache_480_b200 import workloads as wl
+    sc = wl.make_cow_scenario()
+    NB, Hkv, bs, D = sc.num_blocks, sc.num_kv_heads, sc.block_size, sc.head_size
+    bm = pkv.BlockManager(NB, bs, free_order=np.random.default_rng(sc.seed + 1).permutation(NB))
+    kc = torch.full((NB, Hkv, bs, D), float("nan"), dtype=torch.bfloat16, device=device)
+    vc = torch.full_like(kc, float("nan"))
+    pk, pv = wl.cow_prefix_kv(sc, device)
+    pos = 0
+    for p in range(sc.num_prompts):
+        root, L = p * sc.samples, int(sc.prefix_lens[p])
+        bm.allocate(root, L)
+        t = np.arange(L)
+        slots = bm.block_table(root)[t // bs].astype(np.int64) * bs + t % bs
+        pkv.reshape_and_cache(pk[pos:pos + L], pv[pos:pos + L], kc, vc, torch.from_numpy(slots).to(device))
+        pos += L
+        for j in range(1, sc.samples):
+            bm.fork(root, root + j)
+    seqs = np.arange(sc.num_seqs)
+    slots, pairs = bm.append_slots(seqs)     # every sample writes one token this step
+    lens = (sc.prefix_lens[:, None] + np.ones_like(sc.own_tokens)).reshape(-1).astype(np.int32)
+    MB = int(-(-lens.max() // bs))
+    tables, glens = bm.fill_tables(seqs, MB)
+    assert np.array_equal(glens, lens)
+    lay = wl.Layout(name="cow_bf16", dtype="bf16", num_seqs=sc.num_seqs, num_heads=sc.num_heads,
+                    num_kv_heads=Hkv, head_size=D, block_size=bs, num_blocks=NB, scale=sc.scale,
+                    value_scale=1.0, context_lens=lens, block_tables=tables, slot_mapping=slots,
+                    seed=sc.seed, extra=dict(cow_pairs=pairs))
+    gen = torch.Generator(device=device).manual_seed(sc.seed)
+    k_new = torch.randn((sc.num_seqs, Hkv, D), generator=gen, device=device).to(torch.bfloat16)
+    v_new = torch.randn((sc.num_seqs, Hkv, D), generator=gen, device=device).to(torch.bfloat16)
+    ten = dict(q=wl.cow_queries(sc, device), k_cache=kc, v_cache=vc, k_new=k_new, v_new=v_new)
+    return lay, ten, pairs
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("decode_kernel.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_480_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, block_size):
+    """DRAM bytes per decode call from a committed ncu summary, if it still
+    matches the kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    key = f"{workload}/bs{block_size}"
+    e = d.get(key)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_call")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(lay, host, budget_s, max_seqs=None):
+    """Time the oracle on leading sequences of the workload (bounded), repeating
+    until ~budget_s of work; returns (GB/s, seconds, bytes, seqs, threads)."""
+    import oracle
+    S = lay.num_seqs if max_seqs is None else min(max_seqs, lay.num_seqs)
+    sub = lambda a: a[:S]
+    threads = oracle.default_threads()
+    from paged_kv_cache_480_b200 import workloads as wl
+    sublay = wl.Layout(**{**lay.__dict__, "num_seqs": S, "context_lens": sub(lay.context_lens),
+                          "block_tables": sub(lay.block_tables), "slot_mapping": sub(lay.slot_mapping)})
+    nbytes = decode_bytes(sublay)
+    total_t, total_b, reps = 0.0, 0, 0
+    while total_t < budget_s or reps == 0:
+        t0 = time.perf_counter()
+        oracle.paged_attention(host["q"][:S], host["k_cache"], host["v_cache"], sublay.block_tables,
+                               sublay.context_lens, lay.scale, lay.dtype, lay.num_kv_heads,
+                               lay.block_size, nthreads=threads)
+        total_t += time.perf_counter() - t0
+        total_b += nbytes
+        reps += 1
+        if total_t > 2 * budget_s:
+            break
+    return total_b / total_t / 1e9, total_t, total_b, S * reps, threads
+
+
+def host_arrays(ten, dtype):
+    import torch
+    out = {}
+    for k in ("q", "k_cache", "v_cache"):
+        t = ten[k].contiguous().cpu()
+        out[k] = t.numpy() if dtype == "f32" else t.view(torch.int16).numpy().view(np.uint16)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the arms
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """The CPU oracle, as it stands, timed on this host's cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    from paged_kv_cache_480_b200 import workloads as wl
+    name = args.workload
+    if name == "cow_bf16":
+        return {"impl": "reference", "unavailable": "the oracle reference arm runs the decode workloads only"}
+    lay = wl.make_layout(name, block_size=args.block_size)
+    ten = wl.make_tensors(lay, device="cpu", pending_new_token=False)
+    host = host_arrays(ten, lay.dtype)
+    # bounded sample per step: enough sequences for ~1-3 s of oracle work
+    probe_gbs, _, _, _, _ = oracle_sample(lay, host, 0.0, max_seqs=max(1, lay.num_seqs // 16))
+    per_step = max(1, min(lay.num_seqs, int(2.0 * probe_gbs * 1e9 / max(decode_bytes(lay) / lay.num_seqs, 1))))
+    for _ in range(args.warmup):
+        oracle_sample(lay, host, 0.0, max_seqs=per_step)
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        gbs, t, b, seqs, threads = oracle_sample(lay, host, 0.0, max_seqs=per_step)
+        times.append(t)
+        nbytes = b
+    ms = 1e3 * sum(times) / len(times)
+    value = nbytes / (sum(times) / len(times)) / 1e9
+    sample = f"{per_step} of {lay.num_seqs} sequences (all heads) per step"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": name, "block_size": lay.block_size,
+                                            "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import paged_kv_cache_480_b200 as pkv
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    pkv.load_library()
+    lay, ten, pairs = build_workload(args.workload, args.block_size, device)
+    S, H, Hkv, D, bs = lay.num_seqs, lay.num_heads, lay.num_kv_heads, lay.head_size, lay.block_size
+    max_ctx = lay.max_context_len
+    bt = torch.from_numpy(lay.block_tables).to(device)
+    cl = torch.from_numpy(lay.context_lens).to(device)
+    sm = torch.from_numpy(lay.slot_mapping).to(device)
+    pairs_d = torch.from_numpy(np.ascontiguousarray(pairs)).to(device) if pairs is not None and len(pairs) else None
+    out = torch.empty_like(ten["q"])
+    code = {"f32": 0, "f16": 1, "bf16": 2}[lay.dtype]
+    ps = args.partition_size
+    need = pkv.paged_attention_workspace_size(S, H, Hkv, D, bs, max_ctx, code, ps)
+    ws = torch.zeros(need, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    nparts = pkv.paged_attention_partition_size(H, Hkv, bs, max_ctx, ps)
+    split = max_ctx > nparts
+    launches_per_step = 2 + (1 if split else 0) + (1 if pairs_d is not None else 0)
+
+    ev = []
+
+    def step(record=False):
+        if pairs_d is not None:
+            pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], pairs_d, stream=stream)
+        pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm, stream=stream)
+        if record:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                                   max_context_len=max_ctx, partition_size=ps, workspace=ws,
+                                   stream=stream)
+        if record:
+            b.record(stream)
+            ev.append((a, b))
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert pkv.read_device_errors() == 0
+    if world > 1:
+        dist.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    dec_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    errors = pkv.read_device_errors()
+
+    step_bytes = decode_bytes(lay) + cache_write_bytes(lay)
+    if pairs_d is not None:
+        step_bytes += 2 * len(pairs) * 2 * Hkv * bs * D * 2
+    ms_step = ms_total / args.steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = peaks()
+        dec_avg = sum(dec_ms) / len(dec_ms)
+        achieved = decode_bytes(lay) / (dec_avg * 1e-3) / 1e9
+        roof = {"kernel": "paged_attention_decode (decode" + (" + lse merge)" if split else ")"),
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind,
+                "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
+                "traffic": profiled_traffic(lay.name, bs), "algorithmic_bytes": decode_bytes(lay),
+                "avg_call_us": dec_avg * 1e3}
+        result = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                  "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                  "us_per_step": ms_step * 1e3, "seqs_per_s": world * S / (ms_step * 1e-3),
+                  "pct_of_peak": 100 * value / world / peak,
+                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                  "dtype": lay.dtype, "data": "synthetic",
+                  "config": {"workload": lay.name, "num_seqs": S, "num_heads": H,
+                             "num_kv_heads": Hkv, "head_size": D, "block_size": bs,
+                             "num_blocks": lay.num_blocks, "max_context_len": max_ctx,
+                             "mean_context_len": float(lay.context_lens.mean()),
+                             "partition_size": nparts, "split_context": split,
+                             "cow_pairs": 0 if pairs is None else int(len(pairs)),
+                             "step_bytes": step_bytes,
+                             "l2": f"inputs larger than L2: {lay.kv_bytes() / 1e9:.2f} GB of K/V per step",
+                             "parallelism": f"replicas x{world}"},
+                  "roofline": roof, "gpu_launches": launches_per_step * args.steps,
+                  "clocks": clk.summary(), "device_errors": errors}
+        if not args.no_e2e:
+            result["e2e"] = run_e2e(args, lay, ten, pairs, device, ws, step_bytes)
+        if not args.no_cpu_baseline and world == 1:
+            host = host_arrays(ten, lay.dtype)
+            gbs, t, b, seqs, threads = oracle_sample(lay, host, 10.0,
+                                                     max_seqs=max(1, lay.num_seqs // 8))
+            result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                      "sample": f"fp64 oracle over the first {max(1, lay.num_seqs // 8)} "
+                                                f"sequences, repeated: {seqs} sequence-passes in {t:.1f} s"}
+    return result
+
+
+def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
+    """Same step through the C ABI with the step's inputs in pinned host
+    memory: H2D of q, new K/V, slots, tables, lengths (and CoW pairs) and D2H
+    of the output inside the timed region, every step."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    pin = lambda t: t.detach().cpu().pin_memory()
+    h_q, h_k, h_v = pin(ten["q"]), pin(ten["k_new"]), pin(ten["v_new"])
+    h_sm = torch.from_numpy(lay.slot_mapping).pin_memory()
+    h_bt = torch.from_numpy(lay.block_tables).pin_memory()
+    h_cl = torch.from_numpy(lay.context_lens).pin_memory()
+    h_pairs = torch.from_numpy(np.ascontiguousarray(pairs)).pin_memory() if pairs is not None and len(pairs) else None
+    d = {k: torch.empty_like(v, device=device) for k, v in
+         dict(q=h_q, k=h_k, v=h_v, sm=h_sm, bt=h_bt, cl=h_cl).items()}
+    d_pairs = torch.empty_like(h_pairs, device=device) if h_pairs is not None else None
+    out = torch.empty_like(d["q"])
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    stream = torch.cuda.current_stream(device)
+    max_ctx = lay.max_context_len
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_sm, h_bt, h_cl))
+    if h_pairs is not None:
+        h2d += h_pairs.numel() * h_pairs.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+
+    def step():
+        for k, h in (("q", h_q), ("k", h_k), ("v", h_v), ("sm", h_sm), ("bt", h_bt), ("cl", h_cl)):
+            d[k].copy_(h, non_blocking=True)
+        if h_pairs is not None:
+            d_pairs.copy_(h_pairs, non_blocking=True)
+            pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], d_pairs, stream=stream)
+        pkv.reshape_and_cache(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], stream=stream)
+        pkv.paged_attention_decode(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"],
+                                   lay.scale, max_context_len=max_ctx, workspace=ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    return {"value": step_bytes / dt / 1e9, "unit": "GB/s", "us_per_step": dt * 1e6,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

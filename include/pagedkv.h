@@ -1,0 +1,243 @@
+/*
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ *
+ * The library implements the data-parallel hot path of PagedAttention as
+ * the pages describe it:
+ *   - "Efficient Memory Management for Large Language Model Serving with
+ *     PagedAttention" (summary page, xasun.com article 3997), section 2:
+ *     attention whose keys and values sit in non-contiguous, fixed-size
+ *     physical blocks, fetched block by block through a per-sequence block
+ *     table; a KV-cache manager maps logical to physical blocks and
+ *     allocates them on demand; section 1: reference counts plus
+ *     copy-on-write let parallel samples and shared prefixes share blocks.
+ *   - "PyTorch-CUDA-v2.9 image enables PagedAttention" (jsqmd.com 164355),
+ *     PagedAttention section and workflow list: pages of 16 tokens, a page
+ *     table from logical position to physical page, a global page pool,
+ *     each decode step appends the new token's key/value.
+ *   - "GPT-OSS memory management: PagedAttention explained"
+ *     (yongjin360.com 448593), section 2.2: the table tells where token N's
+ *     key/value lives.
+ *
+ * Conventions for every call below
+ *   Layout   caches are [num_blocks][num_kv_heads][block_size][head_size]
+ *            (row-major, contiguous); token t of a sequence lives in block
+ *            block_table[t / block_size] at offset t % block_size; query
+ *            head h reads KV head h / (num_heads / num_kv_heads).  q and out
+ *            are [num_seqs][num_heads][head_size], contiguous.
+ *   Pointers "device" pointers must be CUDA device memory of the current
+ *            device; every device buffer must start on a 16-byte boundary.
+ *   Ownership the caller owns every buffer.  The library allocates no
+ *            device memory and keeps no pointer after a call returns.  The
+ *            block manager owns host memory only (create/destroy).
+ *   Streams  GPU calls are asynchronous on the given cudaStream_t (passed as
+ *            void*, NULL = the legacy default stream); they never
+ *            synchronise, except pkv_read_device_errors.
+ *   Errors   argument errors are found on the host before anything is
+ *            launched and return a status with nothing launched.  A failed
+ *            launch returns PKV_ERR_CUDA.  Conditions only the device can see
+ *            (a block id outside the pool, a slot outside the pool, a context
+ *            longer than the table or than max_context_len) make the kernel
+ *            skip the offending access and set a sticky bit, read with
+ *            pkv_read_device_errors.  No kernel traps.
+ *   Threads  calls are thread-safe as long as concurrent calls use
+ *            different workspaces.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,    /* null pointer, negative size, misaligned buffer ... */
+    PKV_ERR_UNSUPPORTED = 2,    /* outside the supported domain (dtype, head_size, ...) */
+    PKV_ERR_CUDA = 3,           /* a CUDA runtime call or a launch failed */
+    PKV_ERR_OUT_OF_BLOCKS = 4,  /* block manager: not enough free blocks (state unchanged) */
+    PKV_ERR_NOT_FOUND = 5,      /* block manager: unknown sequence id / id already in use */
+    PKV_ERR_WORKSPACE = 6,      /* workspace missing or smaller than required */
+    PKV_ERR_DEVICE_CHECK = 7    /* a device-side check fired (see PKV_DEVERR_*) */
+} pkv_status;
+
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+/* Sticky device-side check bits. */
+#define PKV_DEVERR_BLOCK_ID 1u  /* a block-table entry outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT 2u      /* a slot outside [0, num_blocks * block_size) */
+#define PKV_DEVERR_CONTEXT 4u   /* context_len < 0, > max_blocks_per_seq * block_size or > max_context_len */
+#define PKV_DEVERR_COPY_ID 8u   /* a copy_blocks pair outside [0, num_blocks) */
+#define PKV_DEVERR_WAIT 16u     /* a bounded wait for an asynchronous copy gave up */
+
+const char* pkv_status_string(pkv_status status);
+const char* pkv_version(void);
+
+/* ---------------------------------------------------------------------------
+ * paged_attention_decode -- one decode step of attention for a batch.
+ *
+ * Defines: out[s, h, :] = sum_t softmax_t(scale * q[s,h] . K_s[t]) V_s[t] over
+ * t < context_lens[s], with K_s[t] = k_cache[block_tables[s][t / bs]][h / G]
+ * [t % bs] (V likewise) -- the summary page of the SOSP 2023 paper, section 2
+ * (attention over non-contiguous blocks through the block table) and
+ * section 1 (exact: the output distribution is unchanged).  A sequence with
+ * context_lens[s] == 0 gets an all-zero output.
+ *
+ *   out            device, [num_seqs][num_heads][head_size], dtype (written)
+ *   q              device, [num_seqs][num_heads][head_size], dtype
+ *   k_cache        device, [num_blocks][num_kv_heads][block_size][head_size], dtype
+ *   v_cache        device, same shape as k_cache
+ *   block_tables   device, int32 [num_seqs][max_blocks_per_seq]; entries past
+ *                  ceil(context_len / block_size) are never read
+ *   context_lens   device, int32 [num_seqs]; tokens to attend (includes the
+ *                  step's own token once reshape_and_cache wrote it)
+ *   scale          softmax scale (usually 1/sqrt(head_size))
+ *   num_kv_heads   KV heads; num_heads must be a multiple (G = num_heads /
+ *                  num_kv_heads in {1, 2, 4, 8})
+ *   block_size     tokens per block, 16 or 32
+ *   num_seqs ... max_blocks_per_seq   the sizes above
+ *   max_context_len host-known upper bound of context_lens (> 0); sizes the
+ *                  workspace and picks the split
+ *   dtype          element type of q, caches and out (all the same)
+ *   partition_size tokens per split-context partition: 0 = library choice;
+ *                  otherwise a multiple of block_size, at most 32 *
+ *                  block_size.  Contexts longer than one partition are
+ *                  processed in parallel pieces whose softmax statistics a
+ *                  second kernel merges (log-sum-exp reduction).
+ *   workspace      device scratch of at least
+ *                  paged_attention_workspace_size(...) bytes.  Its first 256
+ *                  bytes hold scheduling counters that must be zero before
+ *                  the first use (paged_attention_workspace_init, or a
+ *                  zero-filled allocation); every call leaves them zero.
+ *                  Calls that run concurrently need separate workspaces.
+ *   stream         cudaStream_t (void*), may be NULL
+ *
+ * Supported: dtype f32/f16/bf16, head_size 64 or 128, block_size 16 or 32,
+ * G in {1, 2, 4, 8}, num_seqs <= 16384.  Anything else: PKV_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------- */
+pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int num_kv_heads,
+                                  int block_size, int num_seqs, int num_heads, int head_size,
+                                  int num_blocks, int max_blocks_per_seq, int max_context_len,
+                                  pkv_dtype dtype, int partition_size, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace paged_attention_decode needs for these sizes (0 on bad
+ * arguments).  partition_size as in paged_attention_decode. */
+size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_size, int block_size, int max_context_len,
+                                      pkv_dtype dtype, int partition_size);
+
+/* The partition size paged_attention_decode uses for these arguments
+ * (partition_size 0 resolved to the library's choice); 0 on bad arguments. */
+int paged_attention_partition_size(int num_heads, int num_kv_heads, int block_size,
+                                   int max_context_len, int partition_size);
+
+/* Zero the scheduling counters of a workspace (asynchronous memset). */
+pkv_status paged_attention_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * reshape_and_cache -- write each new token's key and value into its slot.
+ *
+ * Defines: for every token i with slot = slot_mapping[i] >= 0 and every KV
+ * head g: k_cache[slot / bs][g][slot % bs][:] = key[i][g][:] and likewise
+ * for value; a negative slot means "skip".  A bit copy, no conversion.  The
+ * decode step appends the new token's key/value ("PyTorch-CUDA-v2.9 image
+ * enables PagedAttention", PagedAttention section; workflow list: prefill
+ * writes the input tokens' KV into pages).
+ *
+ *   key, value     device, token i's head g at element i * *_token_stride +
+ *                  g * head_size (strides in elements, multiples of
+ *                  16 bytes / element size)
+ *   k_cache, v_cache device caches (layout above)
+ *   slot_mapping   device, int64 [num_tokens]
+ *   num_blocks     pool size (slots >= num_blocks * block_size are skipped
+ *                  and flag PKV_DEVERR_SLOT)
+ * ------------------------------------------------------------------------- */
+pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_size, int block_size, int num_blocks,
+                             int64_t key_token_stride, int64_t value_token_stride,
+                             pkv_dtype dtype, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * copy_blocks -- the copy-on-write block copy.
+ *
+ * Defines: for every layer l and pair i, block block_mapping[i][1] of
+ * k_caches[l] and v_caches[l] becomes a copy of block block_mapping[i][0]
+ * (summary page of the SOSP 2023 paper, sections 1 and 2: copy-on-write
+ * when parallel samples or shared prefixes diverge).  A bit copy of
+ * block_bytes bytes per block.  Destinations must be distinct and no
+ * destination may also be a source (pairs are copied in parallel).
+ *
+ *   k_caches, v_caches HOST arrays of num_layers device pointers
+ *   block_mapping  device, int64 [num_pairs][2] = (src, dst)
+ *   num_blocks     pool size of every cache (ids outside flag
+ *                  PKV_DEVERR_COPY_ID and are skipped)
+ *   block_bytes    bytes of one block of one cache (num_kv_heads *
+ *                  block_size * head_size * element size), a multiple of 16
+ *   num_layers     1 .. 256
+ * ------------------------------------------------------------------------- */
+pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                       const int64_t* block_mapping, int num_pairs, int num_blocks,
+                       int64_t block_bytes, void* stream);
+
+/* Synchronise the stream, return the sticky device-check bits of the
+ * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
+ * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */
+pkv_status pkv_read_device_errors(void* stream, uint32_t* bits);
+
+/* ---------------------------------------------------------------------------
+ * Host block manager (KV-cache manager of the summary page, section 2; the
+ * global page pool of the PyTorch-CUDA page's workflow list).  Host memory
+ * only; not thread-safe (one manager per thread or external locking).
+ *
+ * Policy: free blocks are handed out first-in first-out from a list whose
+ * initial order is free_order (NULL = 0..num_blocks-1); freed blocks go to
+ * the tail.  Allocation is all-or-nothing: when too few blocks are free the
+ * call returns PKV_ERR_OUT_OF_BLOCKS and changes nothing (the summary page,
+ * section 2: all-or-nothing eviction).  Appending into a shared, partially
+ * filled last block first moves the sequence to a fresh copy and reports
+ * the (src, dst) pair, which the caller passes to copy_blocks before
+ * reshape_and_cache writes the token.
+ * ------------------------------------------------------------------------- */
+typedef struct pkv_block_manager pkv_block_manager;
+
+pkv_status pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                         pkv_block_manager** out);
+void pkv_bm_destroy(pkv_block_manager* bm);
+/* New sequence holding num_tokens tokens (ceil(num_tokens / block_size) blocks). */
+pkv_status pkv_bm_allocate(pkv_block_manager* bm, int64_t seq_id, int num_tokens);
+/* child shares all of parent's blocks (each reference count + 1). */
+pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
+/* Slot of the sequence's next token; cow_src and cow_dst receive the copy to make
+ * first, or -1/-1. */
+pkv_status pkv_bm_append_slot(pkv_block_manager* bm, int64_t seq_id, int64_t* slot,
+                              int32_t* cow_src, int32_t* cow_dst);
+/* append_slot for n sequences in order: slots[n]; cow_pairs[2 * k] for the
+ * k-th copy, *num_cow copies.  Stops at the first failure and returns its
+ * status; *num_done tells how many sequences were served. */
+pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                               int64_t* slots, int64_t* cow_pairs, int* num_cow, int* num_done);
+pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
+/* Copy the sequence's table into out[0 .. capacity); *num_blocks = its length. */
+pkv_status pkv_bm_block_table(const pkv_block_manager* bm, int64_t seq_id, int32_t* out,
+                              int capacity, int* num_blocks);
+/* Tables and lengths of n sequences: tables[n][max_blocks_per_seq] (unused
+ * entries -1), context_lens[n]. */
+pkv_status pkv_bm_fill_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n,
+                              int32_t* tables, int max_blocks_per_seq, int32_t* context_lens);
+int pkv_bm_num_free(const pkv_block_manager* bm);
+int pkv_bm_seq_len(const pkv_block_manager* bm, int64_t seq_id);   /* -1 if unknown */
+int pkv_bm_ref_count(const pkv_block_manager* bm, int32_t block);  /* -1 if out of range */
+/* Written token slots / slots of all blocks in use (0 if none in use). */
+double pkv_bm_utilisation(const pkv_block_manager* bm);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

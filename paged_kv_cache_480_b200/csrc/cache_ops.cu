@@ -1,0 +1,90 @@
+// Cache maintenance kernels: the cache write (each new token's K/V into its
+// slot) and the copy-on-write block copy.  Both are bit copies of 16-byte
+// chunks; neither converts data.
+//
+// reshape_and_cache: "PyTorch-CUDA-v2.9 image enables PagedAttention",
+//   PagedAttention section (each decode step appends the new token's
+//   key/value) and workflow list (prefill writes the tokens' KV into pages).
+// copy_blocks: "Efficient Memory Management for Large Language Model Serving
+//   with PagedAttention" summary page, sections 1 and 2 (reference counts and
+//   copy-on-write for parallel sampling and shared prefixes).
+#include "cache_ops.cuh"
+#include "common.cuh"
+
+namespace pkv {
+
+// One thread per 16-byte chunk of one (token, KV head) row of K and of V.
+__global__ void reshape_and_cache_kernel(const CacheWriteParams p) {
+    const int64_t chunks_per_row = p.row_bytes / 16;
+    const int64_t per_token = (int64_t)p.num_kv_heads * chunks_per_row;
+    const int64_t total = (int64_t)p.num_tokens * per_token;
+    const int64_t pool_slots = (int64_t)p.num_blocks * p.block_size;
+    for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
+         w += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = w / per_token;
+        const int64_t rem = w - i * per_token;
+        const int64_t g = rem / chunks_per_row;
+        const int64_t ch = rem - g * chunks_per_row;
+        const int64_t slot = p.slot_mapping[i];
+        if (slot < 0) continue;
+        if (slot >= pool_slots) {
+            if (rem == 0) flag_error(p.errors, PKV_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / p.block_size, off = slot - blk * p.block_size;
+        const int64_t dst = ((blk * p.num_kv_heads + g) * p.block_size + off) * p.row_bytes + ch * 16;
+        const uint4 kv = *reinterpret_cast<const uint4*>(p.key + i * p.key_stride_bytes +
+                                                         g * p.row_bytes + ch * 16);
+        const uint4 vv = *reinterpret_cast<const uint4*>(p.value + i * p.value_stride_bytes +
+                                                         g * p.row_bytes + ch * 16);
+        *reinterpret_cast<uint4*>(p.k_cache + dst) = kv;
+        *reinterpret_cast<uint4*>(p.v_cache + dst) = vv;
+    }
+}
+
+// grid = (pairs, layers, 2 caches); each CTA copies one block with 16-byte
+// vectors, four loads in flight per thread.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyBlocksParams p) {
+    const int pair = blockIdx.x, layer = blockIdx.y, which = blockIdx.z;
+    const int64_t src = p.block_mapping[2 * (int64_t)pair];
+    const int64_t dst = p.block_mapping[2 * (int64_t)pair + 1];
+    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+        if (threadIdx.x == 0 && layer == 0 && which == 0) flag_error(p.errors, PKV_DEVERR_COPY_ID);
+        return;
+    }
+    unsigned char* base = static_cast<unsigned char*>(which ? p.v[layer] : p.k[layer]);
+    const uint4* s = reinterpret_cast<const uint4*>(base + src * p.block_bytes);
+    uint4* d = reinterpret_cast<uint4*>(base + dst * p.block_bytes);
+    const int64_t n = p.block_bytes / 16;
+    int64_t i = threadIdx.x;
+    for (; i + 3 * blockDim.x < n; i += 4 * blockDim.x) {
+        const uint4 a = s[i], b = s[i + blockDim.x], c = s[i + 2 * blockDim.x],
+                    e = s[i + 3 * blockDim.x];
+        d[i] = a;
+        d[i + blockDim.x] = b;
+        d[i + 2 * blockDim.x] = c;
+        d[i + 3 * blockDim.x] = e;
+    }
+    for (; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cudaStream_t stream) {
+    const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.row_bytes / 16);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    const int64_t cap = (int64_t)num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(const CopyBlocksParams& p, int num_pairs, int num_layers,
+                               cudaStream_t stream) {
+    if (num_pairs == 0 || num_layers == 0) return cudaSuccess;
+    dim3 grid(num_pairs, num_layers, 2);
+    copy_blocks_kernel<<<grid, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,37 @@
+// Parameter blocks and launchers of the cache-maintenance kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+struct CacheWriteParams {
+    const unsigned char* key;
+    const unsigned char* value;
+    unsigned char* k_cache;
+    unsigned char* v_cache;
+    const int64_t* slot_mapping;
+    unsigned int* errors;
+    int64_t key_stride_bytes;    // between tokens
+    int64_t value_stride_bytes;
+    int64_t row_bytes;           // head_size * element size (multiple of 16)
+    int num_tokens, num_kv_heads, block_size, num_blocks;
+};
+
+constexpr int kMaxLayers = 256;
+
+struct CopyBlocksParams {
+    void* k[kMaxLayers];
+    void* v[kMaxLayers];
+    const int64_t* block_mapping;   // [pairs][2]
+    unsigned int* errors;
+    int64_t block_bytes;
+    int64_t num_blocks;
+};
+
+cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_copy_blocks(const CopyBlocksParams& p, int num_pairs, int num_layers,
+                               cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,93 @@
+// Host-side dispatch of the decode and merge kernels over the supported
+// (head_size, block_size, group size) combinations for one element type.
+#pragma once
+
+#include <atomic>
+
+#include "decode_kernel.cuh"
+
+namespace pkv {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxDynSmem = 232448;  // 227 KB opt-in per CTA on sm_100
+
+template <typename T, int D, int BS, int G>
+cudaError_t run_decode(const DecodeParams& p, dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream) {
+    static std::atomic<bool> configured[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    auto kernel = paged_decode_kernel<T, D, BS, G>;
+    if (dev >= 0 && dev < kMaxDevices && !configured[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+        if (e != cudaSuccess) return e;
+        configured[dev].store(true, std::memory_order_release);
+    }
+    kernel<<<grid, block, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+#define PKV_FOR_EACH_SHAPE(X) \
+    X(64, 16, 1) X(64, 16, 2) X(64, 16, 4) X(64, 16, 8)     \
+    X(64, 32, 1) X(64, 32, 2) X(64, 32, 4) X(64, 32, 8)     \
+    X(128, 16, 1) X(128, 16, 2) X(128, 16, 4) X(128, 16, 8) \
+    X(128, 32, 1) X(128, 32, 2) X(128, 32, 4) X(128, 32, 8)
+
+template <typename T>
+cudaError_t dispatch_decode(const DecodeParams& p, int D, int BS, int G, dim3 grid, dim3 block,
+                            size_t smem, cudaStream_t stream) {
+#define PKV_CASE(d, bs, g) \
+    if (D == d && BS == bs && G == g) return run_decode<T, d, bs, g>(p, grid, block, smem, stream);
+    PKV_FOR_EACH_SHAPE(PKV_CASE)
+#undef PKV_CASE
+    return cudaErrorInvalidValue;
+}
+
+// Bytes of one warp's shared-memory region for R stages (0 if unsupported).
+template <typename T>
+uint32_t decode_warp_smem(int D, int BS, int G, int R) {
+#define PKV_CASE(d, bs, g) \
+    if (D == d && BS == bs && G == g) return WarpSmem<T, d, bs, g>::bytes(R);
+    PKV_FOR_EACH_SHAPE(PKV_CASE)
+#undef PKV_CASE
+    return 0;
+}
+
+template <typename T>
+cudaError_t dispatch_merge(const ReduceParams& p, int D, cudaStream_t stream) {
+    dim3 grid(p.num_seqs, (p.num_heads + 3) / 4);
+    if (D == 64) lse_merge_kernel<T, 64><<<grid, 64, 0, stream>>>(p);
+    else if (D == 128) lse_merge_kernel<T, 128><<<grid, 128, 0, stream>>>(p);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace pkv
+
+// One set of entry points per element type (defined in decode_<type>.cu).
+#define PKV_DECLARE_DTYPE(name)                                                                  \
+    namespace pkv {                                                                             \
+    cudaError_t decode_##name(const DecodeParams& p, int D, int BS, int G, dim3 grid, dim3 block, \
+                              size_t smem, cudaStream_t stream);                                \
+    uint32_t warp_smem_##name(int D, int BS, int G, int R);                                     \
+    cudaError_t merge_##name(const ReduceParams& p, int D, cudaStream_t stream);                \
+    }
+
+#define PKV_DEFINE_DTYPE(name, T)                                                               \
+    namespace pkv {                                                                             \
+    cudaError_t decode_##name(const DecodeParams& p, int D, int BS, int G, dim3 grid, dim3 block, \
+                              size_t smem, cudaStream_t stream) {                               \
+        return dispatch_decode<T>(p, D, BS, G, grid, block, smem, stream);                      \
+    }                                                                                           \
+    uint32_t warp_smem_##name(int D, int BS, int G, int R) {                                    \
+        return decode_warp_smem<T>(D, BS, G, R);                                                \
+    }                                                                                           \
+    cudaError_t merge_##name(const ReduceParams& p, int D, cudaStream_t stream) {               \
+        return dispatch_merge<T>(p, D, stream);                                                 \
+    }                                                                                           \
+    }
+
+PKV_DECLARE_DTYPE(f32)
+PKV_DECLARE_DTYPE(f16)
+PKV_DECLARE_DTYPE(bf16)

@@ -1,0 +1,344 @@
+// C-ABI entry points: argument checks on the host, launch planning, and the
+// sticky device-check flag.  Nothing here allocates device memory.
+#include <atomic>
+#include <cstring>
+
+#include "cache_ops.cuh"
+#include "decode_launch.cuh"
+#include "pagedkv.h"
+
+namespace {
+
+__device__ unsigned int g_device_errors;
+
+constexpr int kMaxSeqs = 16384;
+constexpr size_t kSchedBytes = 256;
+
+struct DeviceInfo {
+    std::atomic<int> sms{0};
+    std::atomic<unsigned int*> errors{nullptr};
+};
+DeviceInfo g_devices[pkv::kMaxDevices];
+
+// SM count and device address of the error flag for the current device.
+pkv_status device_info(int* sms, unsigned int** errors) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= pkv::kMaxDevices)
+        return PKV_ERR_CUDA;
+    DeviceInfo& d = g_devices[dev];
+    int n = d.sms.load(std::memory_order_acquire);
+    unsigned int* e = d.errors.load(std::memory_order_acquire);
+    if (n == 0 || e == nullptr) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_device_errors) != cudaSuccess) return PKV_ERR_CUDA;
+        e = static_cast<unsigned int*>(addr);
+        d.sms.store(n, std::memory_order_release);
+        d.errors.store(e, std::memory_order_release);
+    }
+    *sms = n;
+    *errors = e;
+    return PKV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int elem_bytes(pkv_dtype t) { return t == PKV_F32 ? 4 : 2; }
+
+bool valid_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+// Shape checks shared by the workspace query and the launch.
+pkv_status check_shape(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                       int block_size, int max_context_len, int dtype) {
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0)
+        return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (head_size != 64 && head_size != 128) return PKV_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
+    if (num_heads % num_kv_heads != 0) return PKV_ERR_UNSUPPORTED;
+    if (!valid_group(num_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs > kMaxSeqs) return PKV_ERR_UNSUPPORTED;
+    return PKV_OK;
+}
+
+// Tokens per partition.  Requested sizes must be multiples of block_size and
+// at most 32 blocks (one block-table entry per lane).  The library's choice
+// is 16 blocks (32 for groups of 4 or more query heads, whose partial
+// results are larger), or the whole context when it fits in one partition.
+int resolve_partition(int num_heads, int num_kv_heads, int block_size, int max_context_len,
+                      int requested) {
+    const int cap = 32 * block_size;
+    if (requested != 0) {
+        if (requested < 0 || requested % block_size != 0 || requested > cap) return 0;
+        return requested;
+    }
+    const int G = num_heads / num_kv_heads;
+    return (G >= 4 ? 32 : 16) * block_size;
+}
+
+struct WorkspaceLayout {
+    size_t prefix, part_ml, part_acc, total;
+    int max_parts;
+};
+
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                 int max_context_len, int ps) {
+    WorkspaceLayout w;
+    const int ctx = max_context_len > 0 ? max_context_len : 1;
+    w.max_parts = (ctx + ps - 1) / ps;
+    const int G = num_heads / num_kv_heads;
+    const size_t items = (size_t)num_seqs * w.max_parts * num_kv_heads;
+    w.prefix = kSchedBytes;
+    size_t off = round_up(w.prefix + sizeof(int32_t) * (num_seqs + 1), 256);
+    w.part_ml = off;
+    if (w.max_parts > 1) off = round_up(off + items * G * sizeof(float2), 256);
+    w.part_acc = off;
+    if (w.max_parts > 1) off = round_up(off + items * G * head_size * sizeof(float), 256);
+    w.total = off;
+    return w;
+}
+
+uint32_t warp_smem(pkv_dtype t, int D, int BS, int G, int R) {
+    switch (t) {
+        case PKV_F32: return pkv::warp_smem_f32(D, BS, G, R);
+        case PKV_F16: return pkv::warp_smem_f16(D, BS, G, R);
+        default: return pkv::warp_smem_bf16(D, BS, G, R);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status s) {
+    switch (s) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PKV_ERR_CUDA: return "CUDA error";
+        case PKV_ERR_OUT_OF_BLOCKS: return "out of blocks";
+        case PKV_ERR_NOT_FOUND: return "unknown or duplicate sequence id";
+        case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case PKV_ERR_DEVICE_CHECK: return "a device-side check fired";
+    }
+    return "unknown status";
+}
+
+const char* pkv_version(void) { return "pagedkv 0.1 sm_100a"; }
+
+int paged_attention_partition_size(int num_heads, int num_kv_heads, int block_size,
+                                   int max_context_len, int partition_size) {
+    if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return 0;
+    if (block_size != 16 && block_size != 32) return 0;
+    return resolve_partition(num_heads, num_kv_heads, block_size, max_context_len, partition_size);
+}
+
+size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_size, int block_size, int max_context_len,
+                                      pkv_dtype dtype, int partition_size) {
+    if (check_shape(num_seqs, num_heads, num_kv_heads, head_size, block_size, max_context_len,
+                    dtype) != PKV_OK)
+        return 0;
+    const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
+                                     partition_size);
+    if (ps == 0) return 0;
+    return workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps).total;
+}
+
+pkv_status paged_attention_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < kSchedBytes) return PKV_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, kSchedBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int num_kv_heads,
+                                  int block_size, int num_seqs, int num_heads, int head_size,
+                                  int num_blocks, int max_blocks_per_seq, int max_context_len,
+                                  pkv_dtype dtype, int partition_size, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PKV_ERR_INVALID_ARG;
+    pkv_status st = check_shape(num_seqs, num_heads, num_kv_heads, head_size, block_size,
+                                max_context_len, dtype);
+    if (st != PKV_OK) return st;
+    if (num_blocks <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
+    if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(block_tables) || !aligned4(context_lens))
+        return PKV_ERR_INVALID_ARG;
+    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
+                                     partition_size);
+    if (ps == 0) return PKV_ERR_INVALID_ARG;
+    const WorkspaceLayout wl =
+        workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    if ((st = device_info(&sms, &errors)) != PKV_OK) return st;
+
+    const int G = num_heads / num_kv_heads;
+    // Shared memory: per-CTA lengths and prefix sums, then one ring per warp.
+    const uint32_t seq_smem = (uint32_t)round_up(sizeof(int32_t) * (2 * (size_t)num_seqs + 1), 128);
+    int R = 4;
+    uint32_t per_warp = warp_smem(dtype, head_size, block_size, G, R);
+    int W = (int)((pkv::kMaxDynSmem - seq_smem) / per_warp);
+    if (W < 6) {
+        R = 3;
+        per_warp = warp_smem(dtype, head_size, block_size, G, R);
+        W = (int)((pkv::kMaxDynSmem - seq_smem) / per_warp);
+    }
+    if (W > 8) W = 8;
+    if (W < 1) return PKV_ERR_UNSUPPORTED;
+
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    pkv::DecodeParams p;
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.part_acc = reinterpret_cast<float*>(ws + wl.part_acc);
+    p.part_ml = reinterpret_cast<float2*>(ws + wl.part_ml);
+    p.sched = reinterpret_cast<int32_t*>(ws);
+    p.prefix_out = reinterpret_cast<int32_t*>(ws + wl.prefix);
+    p.errors = errors;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.partition_size = ps;
+    p.stages = R;
+    p.warps = W;
+    p.warp_smem = per_warp;
+    p.seq_smem = seq_smem;
+
+    const size_t max_items = (size_t)num_seqs * wl.max_parts * num_kv_heads;
+    size_t ctas = (max_items + W - 1) / W;
+    if (ctas > (size_t)sms) ctas = sms;
+    const size_t smem = seq_smem + (size_t)W * per_warp;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (dtype) {
+        case PKV_F32: e = pkv::decode_f32(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
+        case PKV_F16: e = pkv::decode_f16(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
+        default: e = pkv::decode_bf16(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
+    }
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+    if (wl.max_parts > 1) {
+        pkv::ReduceParams r;
+        r.out = out;
+        r.part_acc = p.part_acc;
+        r.part_ml = p.part_ml;
+        r.prefix = p.prefix_out;
+        r.num_seqs = num_seqs;
+        r.num_heads = num_heads;
+        r.num_kv_heads = num_kv_heads;
+        switch (dtype) {
+            case PKV_F32: e = pkv::merge_f32(r, head_size, s); break;
+            case PKV_F16: e = pkv::merge_f16(r, head_size, s); break;
+            default: e = pkv::merge_bf16(r, head_size, s); break;
+        }
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_size, int block_size, int num_blocks,
+                             int64_t key_token_stride, int64_t value_token_stride,
+                             pkv_dtype dtype, void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    const int eb = elem_bytes(dtype);
+    const int64_t row = (int64_t)head_size * eb;
+    if (row % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    if (key_token_stride < (int64_t)num_kv_heads * head_size ||
+        value_token_stride < (int64_t)num_kv_heads * head_size)
+        return PKV_ERR_INVALID_ARG;
+    if ((key_token_stride * eb) % 16 || (value_token_stride * eb) % 16) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    pkv_status st = device_info(&sms, &errors);
+    if (st != PKV_OK) return st;
+    pkv::CacheWriteParams p;
+    p.key = static_cast<const unsigned char*>(key);
+    p.value = static_cast<const unsigned char*>(value);
+    p.k_cache = static_cast<unsigned char*>(k_cache);
+    p.v_cache = static_cast<unsigned char*>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.errors = errors;
+    p.key_stride_bytes = key_token_stride * eb;
+    p.value_stride_bytes = value_token_stride * eb;
+    p.row_bytes = row;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    if (pkv::launch_reshape_and_cache(p, sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                       const int64_t* block_mapping, int num_pairs, int num_blocks,
+                       int64_t block_bytes, void* stream) {
+    if (num_layers < 0 || num_layers > pkv::kMaxLayers || num_pairs < 0 || num_blocks <= 0 ||
+        block_bytes <= 0 || block_bytes % 16 != 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_pairs == 0 || num_layers == 0) return PKV_OK;
+    if (!k_caches || !v_caches || !block_mapping || (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    if (num_pairs > 65535 || num_layers > 65535) return PKV_ERR_UNSUPPORTED;
+    pkv::CopyBlocksParams p;
+    std::memset(&p, 0, sizeof p);
+    for (int l = 0; l < num_layers; ++l) {
+        if (!k_caches[l] || !v_caches[l] || !aligned16(k_caches[l]) || !aligned16(v_caches[l]))
+            return PKV_ERR_INVALID_ARG;
+        p.k[l] = k_caches[l];
+        p.v[l] = v_caches[l];
+    }
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    pkv_status st = device_info(&sms, &errors);
+    if (st != PKV_OK) return st;
+    p.block_mapping = block_mapping;
+    p.errors = errors;
+    p.block_bytes = block_bytes;
+    p.num_blocks = num_blocks;
+    if (pkv::launch_copy_blocks(p, num_pairs, num_layers, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+pkv_status pkv_read_device_errors(void* stream, uint32_t* bits) {
+    if (!bits) return PKV_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_errors, sizeof v) != cudaSuccess) return PKV_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_device_errors, &zero, sizeof zero) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    *bits = v;
+    return v ? PKV_ERR_DEVICE_CHECK : PKV_OK;
+}
+
+}  // extern "C"
