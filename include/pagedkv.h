@@ -185,6 +185,41 @@ pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_lay
                        const int64_t* block_mapping, int num_pairs, int num_blocks,
                        int64_t block_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * paged_attention_decode_noalloc -- paged_attention_decode without a
+ * workspace argument.  The pages have no counterpart: this entry point only
+ * serves callers that cannot allocate device memory, such as a plug-in
+ * inside a host framework that owns every device allocation through its own
+ * arena, or a latency-critical loop that cannot accept cudaMalloc's implicit
+ * device synchronisation.  The caller still passes the inputs and the output.
+ *
+ * Scratch: one fixed array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) inside the
+ * library, reserved on every GPU that loads the library until the process
+ * exits.  Sizes whose workspace (paged_attention_workspace_size) exceeds it
+ * are rejected with PKV_ERR_WORKSPACE and nothing is launched; all other
+ * argument checks and results are those of paged_attention_decode.  The
+ * call allocates nothing (no cudaMalloc, no cudaFree): it clears the
+ * scheduling counters at the head of the array with an asynchronous memset
+ * on the stream, then launches.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ *
+ * Sharing: every call, on every stream and thread, uses the same array, which
+ * keeps the previous call's contents.  Calls that overlap on the GPU race on
+ * it; serialise them (one stream, or events between streams).
+ * ------------------------------------------------------------------------- */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+pkv_status paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                          const void* v_cache, const int32_t* block_tables,
+                                          const int32_t* context_lens, float scale,
+                                          int num_kv_heads, int block_size, int num_seqs,
+                                          int num_heads, int head_size, int num_blocks,
+                                          int max_blocks_per_seq, int max_context_len,
+                                          pkv_dtype dtype, int partition_size, void* stream);
+
 /* Synchronise the stream, return the sticky device-check bits of the
  * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
  * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */

@@ -60,6 +60,8 @@ def load_library(path=LIB_PATH):
         lib.reshape_and_cache.restype = I
         lib.copy_blocks.argtypes = [P, P, I, P, I, I, I64, P]
         lib.copy_blocks.restype = I
+        lib.paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P]
+        lib.paged_attention_decode_noalloc.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         lib.pkv_read_device_errors.restype = I
         lib.pkv_bm_create.argtypes = [I, I, P, ctypes.POINTER(P)]
@@ -194,6 +196,37 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream, q.device))
     _check(st, "paged_attention_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                   max_context_len=None, partition_size=0, stream=None):
+    """Decode attention using the library's fixed internal scratch instead of
+    a workspace (paged_attention_decode_noalloc in pagedkv.h): for callers
+    that cannot allocate device memory.  Calls on different streams must not
+    overlap; sizes needing more than 16 MiB of scratch raise."""
+    import torch
+    lib = load_library()
+    S, H, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if out.dtype != q.dtype or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("out, q and the caches must share a dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    MB = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = MB * bs
+    st = lib.paged_attention_decode_noalloc(
+        _contig(out, "out"), _contig(q, "q"), _contig(k_cache, "k_cache"), _contig(v_cache, "v_cache"),
+        _contig(block_tables, "block_tables"), _contig(context_lens, "context_lens"),
+        float(scale), Hkv, bs, S, H, D, NB, MB, int(max_context_len), _dtype_code(q),
+        int(partition_size), _stream(stream, q.device))
+    _check(st, "paged_attention_decode_noalloc")
     return out
 
 
