@@ -15,6 +15,8 @@ namespace pkv {
 
 // One thread per 16-byte chunk of one (token, KV head) row of K and of V.
 __global__ void reshape_and_cache_kernel(const CacheWriteParams p) {
+    griddep_wait();
+    griddep_launch();
     const int64_t chunks_per_row = p.row_bytes / 16;
     const int64_t per_token = (int64_t)p.num_kv_heads * chunks_per_row;
     const int64_t total = (int64_t)p.num_tokens * per_token;
@@ -45,6 +47,8 @@ __global__ void reshape_and_cache_kernel(const CacheWriteParams p) {
 // grid = (pairs, layers, 2 caches); each CTA copies one block with 16-byte
 // vectors, four loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyBlocksParams p) {
+    griddep_wait();
+    griddep_launch();
     const int pair = blockIdx.x, layer = blockIdx.y, which = blockIdx.z;
     const int64_t src = p.block_mapping[2 * (int64_t)pair];
     const int64_t dst = p.block_mapping[2 * (int64_t)pair + 1];
@@ -75,16 +79,14 @@ cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cud
     int64_t blocks = (total + threads - 1) / threads;
     const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
-    reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(reshape_and_cache_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, p);
 }
 
 cudaError_t launch_copy_blocks(const CopyBlocksParams& p, int num_pairs, int num_layers,
                                cudaStream_t stream) {
     if (num_pairs == 0 || num_layers == 0) return cudaSuccess;
     dim3 grid(num_pairs, num_layers, 2);
-    copy_blocks_kernel<<<grid, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(copy_blocks_kernel, grid, dim3(256), 0, stream, p);
 }
 
 }  // namespace pkv

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pagedkv.h"
 
 namespace pkv {
@@ -167,6 +169,34 @@ __device__ __forceinline__ int lds32(uint32_t addr) {
 
 __device__ __forceinline__ void flag_error(unsigned int* flags, unsigned int bit) {
     if (flags) atomicOr(flags, bit);
+}
+
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation: it may become resident while its
+// predecessor on the stream finishes, and waits (griddep_wait) for that
+// predecessor's completion and memory before touching global memory.  Each
+// kernel lets its own successor get resident early (griddep_launch).
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Polls of an mbarrier before a wait is declared lost (far beyond any

@@ -18,13 +18,18 @@
 //   grid   = persistent: one CTA per SM, W warps; items beyond the first
 //            per warp come from an atomic counter in the workspace (the last
 //            warp to finish resets it).
-// Arithmetic (all fp32): lane = (token slot u, head h, dim group c); Q lanes
-// share a token row, each holding head_size / Q dims of q (pre-scaled by
-// scale * log2 e) and of the accumulator.  Dot products reduce over the Q
-// lanes with xor shuffles; the online softmax works block-wise in base 2;
-// a whole-sequence item writes the normalised output, a partial one writes
-// (acc, m, l) for the log-sum-exp merge kernel.
+//
+// The arithmetic of a stage is a consumer type:
+//   FmaConsumer  fp32 CUDA-core FMAs (every element type, small groups);
+//   MmaConsumer  tensor-core mma.m16n8k16 for groups of 4-8 query heads with
+//                16-bit elements, where the fp32 FMA issue rate, not HBM,
+//                would bound the kernel.
+// Both keep a base-2 online softmax per head; a whole-sequence item writes
+// the normalised output, a partial one writes (acc, m, l) for the
+// log-sum-exp merge kernel (merge_kernel.cuh).
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -54,17 +59,9 @@ struct DecodeParams {
 template <typename T, int D, int BS, int G>
 struct DecodeShape {
     static constexpr int EPC = Elem<T>::kPerChunk;  // elements per 16-byte chunk
-    static constexpr int NCH = D / EPC;             // chunks per token row
-    static constexpr int Q = (G >= 8) ? 4 : 8;      // lanes per token row
-    static constexpr int CPL = NCH / Q;             // chunks per lane
-    static constexpr int DL = CPL * EPC;            // dims per lane
-    static constexpr int TS = 32 / (Q * G);         // token rows per warp step
-    static constexpr int NSTEP = BS / TS;           // warp steps per block
     static constexpr int ROW = D * (int)sizeof(T);  // bytes per token row
     static constexpr int TILE = BS * ROW;           // bytes per (block, KV head) tile
     static constexpr int QBYTES = G * ROW;          // q rows of one group
-    static_assert(NCH % Q == 0 && CPL >= 1, "head_size too small for the lane layout");
-    static_assert(TS >= 1 && BS % TS == 0, "group size");
 };
 
 struct StageMeta {
@@ -109,11 +106,373 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+constexpr unsigned kFull = 0xffffffffu;
+
+// ===========================================================================
+// fp32 CUDA-core consumer.
+// lane = (token slot u, head h, dim group c); Q lanes share a token row, each
+// holding D / Q dims of q (pre-scaled by scale * log2 e) and of the
+// accumulator; dot products reduce over the Q lanes with xor shuffles.  The 8
+// lanes of a quarter-warp read one 128-byte segment of a row (no bank
+// conflicts).
+// ===========================================================================
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams p) {
+struct FmaConsumer {
+    using S = DecodeShape<T, D, BS, G>;
+    static constexpr int EPC = S::EPC;
+    static constexpr int NCH = D / EPC;             // chunks per token row
+    static constexpr int Q = (G >= 8) ? 4 : 8;      // lanes per token row
+    static constexpr int CPL = NCH / Q;             // chunks per lane
+    static constexpr int DL = CPL * EPC;            // dims per lane
+    static constexpr int TS = 32 / (Q * G);         // token rows per warp step
+    static constexpr int NSTEP = BS / TS;           // warp steps per block
+    static_assert(NCH % Q == 0 && CPL >= 1, "head_size too small for the lane layout");
+    static_assert(TS >= 1 && BS % TS == 0, "group size");
+
+    int c, h, u;
+    float qf[DL], acc[DL];
+    float m_run, l_run;
+
+    __device__ __forceinline__ void init(int lane) {
+        c = lane % Q;
+        h = (lane / Q) % G;
+        u = lane / (Q * G);
+        m_run = -INFINITY;
+        l_run = 0.f;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) qf[d] = acc[d] = 0.f;
+    }
+
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float scale_log2) {
+        const uint4* qrow = reinterpret_cast<const uint4*>(qslot + h * S::ROW);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            float f[EPC];
+            Elem<T>::widen(qrow[c + Q * k], f);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) qf[k * EPC + e] = f[e] * scale_log2;
+        }
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[d] = 0.f;
+        m_run = -INFINITY;
+        l_run = 0.f;
+    }
+
+    __device__ __forceinline__ void block(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float) {
+        float z[NSTEP];
+#pragma unroll
+        for (int i = 0; i < NSTEP; ++i) {
+            const int t = i * TS + u;
+            const uint4* row = reinterpret_cast<const uint4*>(Kt + t * S::ROW);
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                float f[EPC];
+                Elem<T>::widen(row[c + Q * k], f);
+#pragma unroll
+                for (int e = 0; e < EPC; e += 2) {
+                    s0 = fmaf(qf[k * EPC + e], f[e], s0);
+                    s1 = fmaf(qf[k * EPC + e + 1], f[e + 1], s1);
+                }
+            }
+            float sc = s0 + s1;
+#pragma unroll
+            for (int off = 1; off < Q; off <<= 1) sc += __shfl_xor_sync(kFull, sc, off);
+            z[i] = (t < nvalid) ? sc : -INFINITY;
+        }
+        float mb = z[0];
+#pragma unroll
+        for (int i = 1; i < NSTEP; ++i) mb = fmaxf(mb, z[i]);
+#pragma unroll
+        for (int off = Q * G; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+        const float m_new = fmaxf(m_run, mb);   // finite: nvalid > 0
+        const float alpha = ex2(m_run - m_new);
+        l_run *= alpha;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[d] *= alpha;
+#pragma unroll
+        for (int i = 0; i < NSTEP; ++i) {
+            const int t = i * TS + u;
+            if (t < nvalid) {
+                const float pr = ex2(z[i] - m_new);
+                l_run += pr;
+                const uint4* row = reinterpret_cast<const uint4*>(Vt + t * S::ROW);
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) {
+                    float f[EPC];
+                    Elem<T>::widen(row[c + Q * k], f);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) acc[k * EPC + e] = fmaf(pr, f[e], acc[k * EPC + e]);
+                }
+            }
+        }
+        m_run = m_new;
+    }
+
+    __device__ __forceinline__ void finish(const StageMeta& mt, const DecodeParams& p) {
+        float lt = l_run;
+#pragma unroll
+        for (int off = Q * G; off < 32; off <<= 1) {
+            lt += __shfl_xor_sync(kFull, lt, off);
+#pragma unroll
+            for (int d = 0; d < DL; ++d) acc[d] += __shfl_xor_sync(kFull, acc[d], off);
+        }
+        if (u != 0) return;
+        if (mt.flags & kWhole) {
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) +
+                                                   ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + h) * D);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                float f[EPC];
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) f[e] = acc[k * EPC + e] * inv;
+                orow[c + Q * k] = Elem<T>::narrow(f);
+            }
+        } else {
+            float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + h) * D);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int e = 0; e < EPC; e += 4)
+                    prow[((c + Q * k) * EPC + e) / 4] =
+                        make_float4(acc[k * EPC + e], acc[k * EPC + e + 1], acc[k * EPC + e + 2],
+                                    acc[k * EPC + e + 3]);
+            if (c == 0) p.part_ml[(size_t)mt.item * G + h] = make_float2(m_run, lt);
+        }
+    }
+};
+
+// ===========================================================================
+// Tensor-core consumer (mma.sync m16n8k16, fp32 accumulate) for 16-bit
+// elements and G in {4, 8}.  Per 16-token slice of a block:
+//   S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]       (D/16 MMAs)
+//   O^T[D x 8 heads]     += V^T[D x 16 tok] . P^T[16 x 8] (D/16 MMAs)
+// Lane = (r = lane / 4, c = lane % 4).  The contraction index of an MMA may
+// be any fixed permutation of the head dims (resp. tokens) as long as both
+// operands use it, so every lane loads whole 16-byte chunks of the tile with
+// plain shared loads:
+//   QK step (j, hf): k-slots (2c, 2c+1) <-> dims 8(4j+c) + 4hf + {0,1},
+//                    k-slots (2c+8, 2c+9) <-> dims 8(4j+c) + 4hf + {2,3};
+//   PV tile m: row r <-> dim r*D/8 + 2m, row r+8 <-> dim r*D/8 + 2m + 1,
+//              k-slot i <-> token i; V^T pairs of adjacent tokens are
+//              assembled with byte permutes.
+// P is rounded to the element type for the second MMA and the softmax sums
+// use the rounded values.  Heads >= G of the 8 MMA columns are zero padding.
+// ===========================================================================
+template <typename T, int D, int BS, int G>
+struct MmaConsumer {
+    using S = DecodeShape<T, D, BS, G>;
+    static_assert(sizeof(T) == 2, "tensor-core consumer needs 16-bit elements");
+    static_assert(G == 4 || G == 8, "tensor-core consumer serves groups of 4 or 8 heads");
+    static constexpr int KJ = D / 32;      // 16-byte chunks per lane per K row
+    static constexpr int MT = D / 16;      // PV MMAs (row tiles of 16 dims)
+    static constexpr int VCH = D / 64;     // 16-byte chunks per lane per V row (D/8 dims)
+    static_assert(D % 64 == 0, "head_size 64 or 128");
+
+    int r, c;
+    uint32_t qf[KJ][4];                    // Q^T fragments (b0, b1 for hf = 0, 1)
+    float o[MT][4];                        // O^T accumulators
+    float m0, m1, l0, l1;                  // heads 2c, 2c+1
+
+    __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            asm volatile(
+                "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+                "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        } else {
+            asm volatile(
+                "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+                "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+
+    __device__ __forceinline__ static uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+        uint32_t d;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+        return d;
+    }
+
+    __device__ __forceinline__ static float lo_f(uint32_t w) {
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) return __uint_as_float(w << 16);
+        else return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+    }
+    __device__ __forceinline__ static float hi_f(uint32_t w) {
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) return __uint_as_float(w & 0xffff0000u);
+        else return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    }
+
+    __device__ __forceinline__ void init(int lane) {
+        r = lane >> 2;
+        c = lane & 3;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KJ; ++j) qf[j][0] = qf[j][1] = qf[j][2] = qf[j][3] = 0u;
+    }
+
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float) {
+        // B operand: column n = head r; rows = permuted dims of chunk 4j + c.
+#pragma unroll
+        for (int j = 0; j < KJ; ++j) {
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (r < G) w = reinterpret_cast<const uint4*>(qslot + r * S::ROW)[4 * j + c];
+            qf[j][0] = w.x;
+            qf[j][1] = w.y;
+            qf[j][2] = w.z;
+            qf[j][3] = w.w;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void slice(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float scale_log2) {
+        // ---- S^T = K . Q^T ----
+        const uint4* k0 = reinterpret_cast<const uint4*>(Kt + r * S::ROW);
+        const uint4* k8 = reinterpret_cast<const uint4*>(Kt + (r + 8) * S::ROW);
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < KJ; ++j) {
+            const uint4 a = k0[4 * j + c];
+            const uint4 b = k8[4 * j + c];
+            mma(sc, a.x, b.x, a.y, b.y, qf[j][0], qf[j][1]);
+            mma(sc, a.z, b.z, a.w, b.w, qf[j][2], qf[j][3]);
+        }
+        // sc: [tok r][head 2c], [tok r][2c+1], [tok r+8][2c], [tok r+8][2c+1]
+        const bool v0 = r < nvalid, v8 = r + 8 < nvalid;
+        const float z0 = v0 ? sc[0] * scale_log2 : -INFINITY;
+        const float z1 = v0 ? sc[1] * scale_log2 : -INFINITY;
+        const float z2 = v8 ? sc[2] * scale_log2 : -INFINITY;
+        const float z3 = v8 ? sc[3] * scale_log2 : -INFINITY;
+        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);   // finite: nvalid > 0
+        const float al0 = ex2(m0 - n0), al1 = ex2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const uint32_t pk_lo = Elem<T>::pack2(ex2(z0 - n0), ex2(z1 - n1));   // token r
+        const uint32_t pk_hi = Elem<T>::pack2(ex2(z2 - n0), ex2(z3 - n1));   // token r + 8
+        l0 = l0 * al0 + lo_f(pk_lo) + lo_f(pk_hi);
+        l1 = l1 * al1 + hi_f(pk_lo) + hi_f(pk_hi);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            o[m][0] *= al0;
+            o[m][2] *= al0;
+            o[m][1] *= al1;
+            o[m][3] *= al1;
+        }
+        // ---- B = P^T: lane (r, c) needs P[head r][tokens 2c, 2c+1, 2c+8, 2c+9] ----
+        const int src0 = (2 * c) * 4 + (r >> 1), src1 = src0 + 4;
+        const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+        const uint32_t x0 = __shfl_sync(kFull, pk_lo, src0), x1 = __shfl_sync(kFull, pk_lo, src1);
+        const uint32_t y0 = __shfl_sync(kFull, pk_hi, src0), y1 = __shfl_sync(kFull, pk_hi, src1);
+        const uint32_t pb0 = prmt(x0, x1, sel), pb1 = prmt(y0, y1, sel);
+        // ---- O^T += V^T . P^T ----
+        uint32_t w[4][4 * VCH];   // rows 2c, 2c+1, 2c+8, 2c+9; words = dim pairs
+        const int rows[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4* vr = reinterpret_cast<const uint4*>(Vt + rows[i] * S::ROW) + r * VCH;
+            const bool ok = rows[i] < nvalid;
+#pragma unroll
+            for (int ch = 0; ch < VCH; ++ch) {
+                uint4 v = vr[ch];
+                if (!ok) v = make_uint4(0u, 0u, 0u, 0u);   // masked tokens may hold NaN
+                w[i][4 * ch + 0] = v.x;
+                w[i][4 * ch + 1] = v.y;
+                w[i][4 * ch + 2] = v.z;
+                w[i][4 * ch + 3] = v.w;
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const uint32_t a0 = prmt(w[0][m], w[1][m], 0x5410u);
+            const uint32_t a1 = prmt(w[0][m], w[1][m], 0x7632u);
+            const uint32_t a2 = prmt(w[2][m], w[3][m], 0x5410u);
+            const uint32_t a3 = prmt(w[2][m], w[3][m], 0x7632u);
+            mma(o[m], a0, a1, a2, a3, pb0, pb1);
+        }
+    }
+
+    __device__ __forceinline__ void block(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float scale_log2) {
+#pragma unroll
+        for (int sl = 0; sl < BS / 16; ++sl) {
+            const int nv = nvalid - 16 * sl;
+            if (nv <= 0) break;
+            slice(Kt + sl * 16 * S::ROW, Vt + sl * 16 * S::ROW, nv, scale_log2);
+        }
+    }
+
+    __device__ __forceinline__ void finish(const StageMeta& mt, const DecodeParams& p) {
+        float t0 = l0, t1 = l1;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            t0 += __shfl_xor_sync(kFull, t0, off);
+            t1 += __shfl_xor_sync(kFull, t1, off);
+        }
+        // lane (r, c) holds dims [r*D/8, (r+1)*D/8) of heads 2c, 2c+1
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * c + e;
+            if (head >= G) continue;
+            const float lt = e ? t1 : t0;
+            if (mt.flags & kWhole) {
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                uint32_t words[MT];
+#pragma unroll
+                for (int m = 0; m < MT; ++m) words[m] = Elem<T>::pack2(o[m][e] * inv, o[m][2 + e] * inv);
+                uint4* orow = reinterpret_cast<uint4*>(
+                    reinterpret_cast<T*>(p.out) +
+                    ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + head) * D + r * (D / 8));
+#pragma unroll
+                for (int ch = 0; ch < VCH; ++ch)
+                    orow[ch] = make_uint4(words[4 * ch], words[4 * ch + 1], words[4 * ch + 2],
+                                          words[4 * ch + 3]);
+            } else {
+                float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + head) * D +
+                                                         r * (D / 8));
+#pragma unroll
+                for (int m = 0; m < MT; m += 2)
+                    prow[m / 2] = make_float4(o[m][e], o[m][2 + e], o[m + 1][e], o[m + 1][2 + e]);
+                if (r == 0)
+                    p.part_ml[(size_t)mt.item * G + head] = make_float2(e ? m1 : m0, lt);
+            }
+        }
+    }
+};
+
+template <typename T, int G>
+struct UseMma {
+    static constexpr bool value = sizeof(T) == 2 && (G == 4 || G == 8);
+};
+
+template <typename T, int D, int BS, int G>
+using ConsumerFor = typename std::conditional<UseMma<T, G>::value, MmaConsumer<T, D, BS, G>,
+                                              FmaConsumer<T, D, BS, G>>::type;
+
+// ===========================================================================
+// The kernel: prologue, producer (bulk-copy ring) and consumer loop.
+// ===========================================================================
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams p) {
     using S = DecodeShape<T, D, BS, G>;
     using L = WarpSmem<T, D, BS, G>;
-    constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ __align__(128) unsigned char smem[];
 
     const int nseq = p.num_seqs;
@@ -128,6 +487,11 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
     const uint32_t bar0 = smem_addr(wb + L::bars(R));
     const int PS = p.partition_size;
 
+    if (lane == 0)
+        for (int st = 0; st < R; ++st) mbar_init(bar0 + 8 * st, 1);
+    fence_mbar_init();
+    griddep_wait();      // inputs may come from the previous kernel on the stream
+
     // ---- lengths and partition prefix sums (every CTA; CTA 0 publishes) ----
     for (int i = threadIdx.x; i < nseq; i += blockDim.x) {
         int len = p.context_lens[i];
@@ -137,9 +501,6 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
         }
         s_len[i] = len;
     }
-    if (lane == 0)
-        for (int st = 0; st < R; ++st) mbar_init(bar0 + 8 * st, 1);
-    fence_mbar_init();
     __syncthreads();
     if (warp == 0) {
         int carry = 0;
@@ -149,17 +510,18 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
             int incl = n;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(FULL, incl, off);
+                const int v = __shfl_up_sync(kFull, incl, off);
                 if (lane >= off) incl += v;
             }
             if (i < nseq) s_pre[i] = carry + incl - n;
-            carry += __shfl_sync(FULL, incl, 31);
+            carry += __shfl_sync(kFull, incl, 31);
         }
         if (lane == 0) s_pre[nseq] = carry;
     }
     __syncthreads();
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i <= nseq; i += blockDim.x) p.prefix_out[i] = s_pre[i];
+    griddep_launch();    // the merge kernel may get resident; it waits for our completion
 
     const int Hkv = p.num_kv_heads;
     const int n_items = s_pre[nseq] * Hkv;
@@ -193,7 +555,7 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
     auto next_index = [&]() -> int {
         int v = 0;
         if (lane == 0) v = atomicAdd(p.sched, 1) + NW;
-        return __shfl_sync(FULL, v, 0);
+        return __shfl_sync(kFull, v, 0);
     };
 
     // ---- producer state ----
@@ -213,7 +575,7 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
     auto issue = [&]() {
         if (P.idx >= n_items) return;
         const int st = issue_st;
-        const int phys = __shfl_sync(FULL, P.tbl, pj & 31);
+        const int phys = __shfl_sync(kFull, P.tbl, pj & 31);
         int nvalid = min(max(P.ntok - pj * BS, 0), BS);
         const bool bad = nvalid > 0 && (phys < 0 || phys >= p.num_blocks);
         if (bad) nvalid = 0;
@@ -251,14 +613,9 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
         }
     };
 
-    // ---- consumer state ----
-    const int c = lane % S::Q;
-    const int h = (lane / S::Q) % G;
-    const int u = lane / (S::Q * G);
-    float qf[S::DL], acc[S::DL];
-    float m_run = -INFINITY, l_run = 0.f;
-#pragma unroll
-    for (int d = 0; d < S::DL; ++d) qf[d] = acc[d] = 0.f;
+    // ---- consumer ----
+    ConsumerFor<T, D, BS, G> cons;
+    cons.init(lane);
 
     for (int i = 0; i < R; ++i) issue();
     int cons_st = 0;
@@ -274,107 +631,12 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
             break;
         }
         const StageMeta mt = meta[cons_st];
-        if (mt.flags & kFirst) {
-            const uint4* qrow = reinterpret_cast<const uint4*>(qbuf + mt.qslot * S::QBYTES + h * S::ROW);
-#pragma unroll
-            for (int k = 0; k < S::CPL; ++k) {
-                float f[S::EPC];
-                Elem<T>::widen(qrow[c + S::Q * k], f);
-#pragma unroll
-                for (int e = 0; e < S::EPC; ++e) qf[k * S::EPC + e] = f[e] * p.scale_log2;
-            }
-#pragma unroll
-            for (int d = 0; d < S::DL; ++d) acc[d] = 0.f;
-            m_run = -INFINITY;
-            l_run = 0.f;
-        }
-        const int nvalid = mt.nvalid;
-        if (nvalid > 0) {
+        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, p.scale_log2);
+        if (mt.nvalid > 0) {
             const unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
-            const unsigned char* Vt = Kt + S::TILE;
-            float z[S::NSTEP];
-#pragma unroll
-            for (int i = 0; i < S::NSTEP; ++i) {
-                const int t = i * S::TS + u;
-                const uint4* row = reinterpret_cast<const uint4*>(Kt + t * S::ROW);
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                for (int k = 0; k < S::CPL; ++k) {
-                    float f[S::EPC];
-                    Elem<T>::widen(row[c + S::Q * k], f);
-#pragma unroll
-                    for (int e = 0; e < S::EPC; e += 2) {
-                        s0 = fmaf(qf[k * S::EPC + e], f[e], s0);
-                        s1 = fmaf(qf[k * S::EPC + e + 1], f[e + 1], s1);
-                    }
-                }
-                float sc = s0 + s1;
-#pragma unroll
-                for (int off = 1; off < S::Q; off <<= 1) sc += __shfl_xor_sync(FULL, sc, off);
-                z[i] = (t < nvalid) ? sc : -INFINITY;
-            }
-            float mb = z[0];
-#pragma unroll
-            for (int i = 1; i < S::NSTEP; ++i) mb = fmaxf(mb, z[i]);
-#pragma unroll
-            for (int off = S::Q * G; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(FULL, mb, off));
-            const float m_new = fmaxf(m_run, mb);   // finite: nvalid > 0
-            const float alpha = ex2(m_run - m_new);
-            l_run *= alpha;
-#pragma unroll
-            for (int d = 0; d < S::DL; ++d) acc[d] *= alpha;
-#pragma unroll
-            for (int i = 0; i < S::NSTEP; ++i) {
-                const int t = i * S::TS + u;
-                if (t < nvalid) {
-                    const float pr = ex2(z[i] - m_new);
-                    l_run += pr;
-                    const uint4* row = reinterpret_cast<const uint4*>(Vt + t * S::ROW);
-#pragma unroll
-                    for (int k = 0; k < S::CPL; ++k) {
-                        float f[S::EPC];
-                        Elem<T>::widen(row[c + S::Q * k], f);
-#pragma unroll
-                        for (int e = 0; e < S::EPC; ++e)
-                            acc[k * S::EPC + e] = fmaf(pr, f[e], acc[k * S::EPC + e]);
-                    }
-                }
-            }
-            m_run = m_new;
+            cons.block(Kt, Kt + S::TILE, mt.nvalid, p.scale_log2);
         }
-        if (mt.flags & kLast) {
-            float lt = l_run;
-#pragma unroll
-            for (int off = S::Q * G; off < 32; off <<= 1) {
-                lt += __shfl_xor_sync(FULL, lt, off);
-#pragma unroll
-                for (int d = 0; d < S::DL; ++d) acc[d] += __shfl_xor_sync(FULL, acc[d], off);
-            }
-            if (u == 0) {
-                if (mt.flags & kWhole) {
-                    const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                    uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) +
-                                                           ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + h) * D);
-#pragma unroll
-                    for (int k = 0; k < S::CPL; ++k) {
-                        float f[S::EPC];
-#pragma unroll
-                        for (int e = 0; e < S::EPC; ++e) f[e] = acc[k * S::EPC + e] * inv;
-                        orow[c + S::Q * k] = Elem<T>::narrow(f);
-                    }
-                } else {
-                    float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + h) * D);
-#pragma unroll
-                    for (int k = 0; k < S::CPL; ++k)
-#pragma unroll
-                        for (int e = 0; e < S::EPC; e += 4)
-                            prow[((c + S::Q * k) * S::EPC + e) / 4] =
-                                make_float4(acc[k * S::EPC + e], acc[k * S::EPC + e + 1],
-                                            acc[k * S::EPC + e + 2], acc[k * S::EPC + e + 3]);
-                    if (c == 0) p.part_ml[(size_t)mt.item * G + h] = make_float2(m_run, lt);
-                }
-            }
-        }
+        if (mt.flags & kLast) cons.finish(mt, p);
         __syncwarp();
         ++consumed;
         if (++cons_st == R) { cons_st = 0; phase ^= 1u; }
@@ -390,59 +652,6 @@ __global__ void __launch_bounds__(256, 1) paged_decode_kernel(const DecodeParams
             atomicExch(p.sched + 1, 0);
         }
     }
-}
-
-// ---------------------------------------------------------------------------
-// Log-sum-exp merge of the partitions of every sequence that has more than
-// one (the exact identity: with M = max_p m_p and w_p = 2^(m_p - M),
-// out = sum_p w_p acc_p / sum_p w_p l_p).  One CTA per (sequence, group of
-// 4 query heads); each thread owns 4 dims of one head.
-// ---------------------------------------------------------------------------
-struct ReduceParams {
-    void* out;
-    const float* part_acc;
-    const float2* part_ml;
-    const int32_t* prefix;
-    int num_seqs, num_heads, num_kv_heads;
-};
-
-template <typename T, int D>
-__global__ void __launch_bounds__(D) lse_merge_kernel(const ReduceParams p) {
-    const int s = blockIdx.x;
-    const int np = p.prefix[s + 1] - p.prefix[s];
-    if (np <= 1) return;
-    const int G = p.num_heads / p.num_kv_heads;
-    const int h = blockIdx.y * 4 + threadIdx.x / (D / 4);
-    if (h >= p.num_heads) return;
-    const int d4 = threadIdx.x % (D / 4);
-    const int g = h / G, hh = h % G;
-    const int base = p.prefix[s];
-    float M = -INFINITY;
-    for (int q = 0; q < np; ++q) {
-        const size_t item = (size_t)(base + q) * p.num_kv_heads + g;
-        M = fmaxf(M, p.part_ml[item * G + hh].x);
-    }
-    float den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-        for (int q = 0; q < np; ++q) {
-            const size_t item = (size_t)(base + q) * p.num_kv_heads + g;
-            const float2 ml = p.part_ml[item * G + hh];
-            if (ml.x == -INFINITY) continue;
-            const float w = ex2(ml.x - M);
-            den = fmaf(w, ml.y, den);
-            const float4 a = reinterpret_cast<const float4*>(p.part_acc + (item * G + hh) * D)[d4];
-            num.x = fmaf(w, a.x, num.x);
-            num.y = fmaf(w, a.y, num.y);
-            num.z = fmaf(w, a.z, num.z);
-            num.w = fmaf(w, a.w, num.w);
-        }
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    float f[4] = {num.x * inv, num.y * inv, num.z * inv, num.w * inv};
-    T* o = reinterpret_cast<T*>(p.out) + ((size_t)s * p.num_heads + h) * D + d4 * 4;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = static_cast<T>(f[e]);
 }
 
 }  // namespace pkv

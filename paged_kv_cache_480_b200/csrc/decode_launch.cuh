@@ -5,6 +5,7 @@
 #include <atomic>
 
 #include "decode_kernel.cuh"
+#include "merge_kernel.cuh"
 
 namespace pkv {
 
@@ -24,8 +25,7 @@ cudaError_t run_decode(const DecodeParams& p, dim3 grid, dim3 block, size_t smem
         if (e != cudaSuccess) return e;
         configured[dev].store(true, std::memory_order_release);
     }
-    kernel<<<grid, block, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kernel, grid, block, smem, stream, p);
 }
 
 #define PKV_FOR_EACH_SHAPE(X) \
@@ -56,11 +56,11 @@ uint32_t decode_warp_smem(int D, int BS, int G, int R) {
 
 template <typename T>
 cudaError_t dispatch_merge(const ReduceParams& p, int D, cudaStream_t stream) {
-    dim3 grid(p.num_seqs, (p.num_heads + 3) / 4);
-    if (D == 64) lse_merge_kernel<T, 64><<<grid, 64, 0, stream>>>(p);
-    else if (D == 128) lse_merge_kernel<T, 128><<<grid, 128, 0, stream>>>(p);
-    else return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    const size_t smem = sizeof(float2) * (size_t)p.max_parts;
+    const dim3 grid(p.num_seqs, p.num_heads);
+    if (D == 64) return launch_pdl(lse_merge_kernel<T, 64>, grid, dim3(128), smem, stream, p);
+    if (D == 128) return launch_pdl(lse_merge_kernel<T, 128>, grid, dim3(128), smem, stream, p);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace pkv
