@@ -101,9 +101,10 @@ const char* pkv_version(void);
  *   max_context_len host-known upper bound of context_lens (> 0); sizes the
  *                  workspace and picks the split
  *   dtype          element type of q, caches and out (all the same)
- *   partition_size tokens per split-context partition: 0 = library choice;
- *                  otherwise a multiple of block_size, at most 32 *
- *                  block_size.  Contexts longer than one partition are
+ *   partition_size tokens per split-context partition: 0 = library choice
+ *                  (a per-call size between 8 and 16 blocks, 16 and 32
+ *                  for G >= 4); otherwise a multiple of block_size, at
+ *                  most 32 * block_size.  Contexts longer than one partition are
  *                  processed in parallel pieces whose softmax statistics a
  *                  second kernel merges (log-sum-exp reduction).
  *   workspace      device scratch of at least
@@ -131,8 +132,11 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_he
                                       int head_size, int block_size, int max_context_len,
                                       pkv_dtype dtype, int partition_size);
 
-/* The partition size paged_attention_decode uses for these arguments
- * (partition_size 0 resolved to the library's choice); 0 on bad arguments. */
+/* The smallest partition size paged_attention_decode may use for these
+ * arguments: the requested size, or for partition_size 0 the lower end of
+ * the library's range (the kernel then picks, per call, a block multiple
+ * between this and twice this that keeps the last round of work items full).
+ * Contexts up to this length are never split.  0 on bad arguments. */
 int paged_attention_partition_size(int num_heads, int num_kv_heads, int block_size,
                                    int max_context_len, int partition_size);
 

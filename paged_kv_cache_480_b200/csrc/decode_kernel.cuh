@@ -50,6 +50,7 @@ struct DecodeParams {
     float scale_log2;       // scale * log2(e)
     int num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int partition_size;     // PS tokens, a multiple of block_size, <= 32 blocks
+    int partition_min;      // > 0: choose PS in [partition_min, partition_size] on the device
     int stages;             // R
     int warps;              // W consumer warps per CTA
     uint32_t warp_smem;     // bytes of one warp's region
@@ -467,6 +468,48 @@ using ConsumerFor = typename std::conditional<UseMma<T, G>::value, MmaConsumer<T
                                               FmaConsumer<T, D, BS, G>>::type;
 
 // ===========================================================================
+// Partition size for the call, chosen identically by every CTA.  With NW
+// warps and n items of equal size the step lasts ceil(n / NW) item-times
+// while the work is n / NW of them: a last round that is only partly full
+// leaves warps idle.  Among the block multiples in [partition_min,
+// partition_size], take the largest whose fill ratio (n/NW) / ceil(n/NW) is
+// within 0.02 of the best.
+// ===========================================================================
+constexpr int kMaxPartitionCandidates = 33;
+
+__device__ __forceinline__ int choose_partition(const int* s_len, int nseq, const DecodeParams& p,
+                                                int bs) {
+    __shared__ int s_count[kMaxPartitionCandidates];
+    __shared__ int s_choice;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int nc = min((p.partition_size - p.partition_min) / bs + 1, kMaxPartitionCandidates);
+    for (int j = warp; j < nc; j += nwarps) {
+        const int ps = p.partition_size - j * bs;
+        int n = 0;
+        for (int i = lane; i < nseq; i += 32) n += max(1, (s_len[i] + ps - 1) / ps);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(kFull, n, off);
+        if (lane == 0) s_count[j] = n;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const float nw = (float)(gridDim.x * p.warps);
+        float fill[kMaxPartitionCandidates];
+        float best = 0.f;
+        for (int j = 0; j < nc; ++j) {
+            const float x = (float)s_count[j] * p.num_kv_heads / nw;
+            fill[j] = x / ceilf(x);
+            best = fmaxf(best, fill[j]);
+        }
+        int pick = 0;
+        while (fill[pick] < best - 0.02f) ++pick;
+        s_choice = p.partition_size - pick * bs;
+    }
+    __syncthreads();
+    return s_choice;
+}
+
+// ===========================================================================
 // The kernel: prologue, producer (bulk-copy ring) and consumer loop.
 // ===========================================================================
 template <typename T, int D, int BS, int G>
@@ -485,7 +528,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
     unsigned char* qbuf = wb + L::qbuf(R);
     StageMeta* meta = reinterpret_cast<StageMeta*>(wb + L::meta(R));
     const uint32_t bar0 = smem_addr(wb + L::bars(R));
-    const int PS = p.partition_size;
+    int PS = p.partition_size;
 
     if (lane == 0)
         for (int st = 0; st < R; ++st) mbar_init(bar0 + 8 * st, 1);
@@ -502,6 +545,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         s_len[i] = len;
     }
     __syncthreads();
+    if (p.partition_min > 0) PS = choose_partition(s_len, nseq, p, BS);
     if (warp == 0) {
         int carry = 0;
         for (int base = 0; base < nseq; base += 32) {

@@ -10,7 +10,7 @@
 namespace pkv {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxDynSmem = 232448;  // 227 KB opt-in per CTA on sm_100
+constexpr int kMaxDynSmem = 232448 - 1024;  // 227 KB opt-in per CTA on sm_100, less static smem
 
 template <typename T, int D, int BS, int G>
 cudaError_t run_decode(const DecodeParams& p, dim3 grid, dim3 block, size_t smem,

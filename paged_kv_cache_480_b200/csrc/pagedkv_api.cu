@@ -66,17 +66,24 @@ pkv_status check_shape(int num_seqs, int num_heads, int num_kv_heads, int head_s
 
 // Tokens per partition.  Requested sizes must be multiples of block_size and
 // at most 32 blocks (one block-table entry per lane).  The library's choice
-// is 16 blocks (32 for groups of 4 or more query heads, whose partial
-// results are larger), or the whole context when it fits in one partition.
+// (requested == 0) is a range: the kernel picks, per call, a block multiple
+// between half and all of 16 blocks (32 for groups of 4 or more query heads,
+// whose partial results are larger) so that the last round of work items
+// keeps the warps busy.  Returns the smallest size the call may use (which
+// sizes the workspace) and, through *largest, the largest.
 int resolve_partition(int num_heads, int num_kv_heads, int block_size, int max_context_len,
-                      int requested) {
+                      int requested, int* largest = nullptr) {
+    (void)max_context_len;
     const int cap = 32 * block_size;
     if (requested != 0) {
         if (requested < 0 || requested % block_size != 0 || requested > cap) return 0;
+        if (largest) *largest = requested;
         return requested;
     }
     const int G = num_heads / num_kv_heads;
-    return (G >= 4 ? 32 : 16) * block_size;
+    const int hi = (G >= 4 ? 32 : 16) * block_size;
+    if (largest) *largest = hi;
+    return hi / 2;
 }
 
 struct WorkspaceLayout {
@@ -173,8 +180,9 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
         !aligned4(block_tables) || !aligned4(context_lens))
         return PKV_ERR_INVALID_ARG;
     if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    int ps_hi = 0;
     const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
-                                     partition_size);
+                                     partition_size, &ps_hi);
     if (ps == 0) return PKV_ERR_INVALID_ARG;
     const WorkspaceLayout wl =
         workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps);
@@ -203,7 +211,7 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
     if (W < 1) return PKV_ERR_UNSUPPORTED;
 
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    pkv::DecodeParams p;
+    pkv::DecodeParams p{};
     p.out = out;
     p.q = q;
     p.k_cache = k_cache;
@@ -222,7 +230,9 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
     p.num_blocks = num_blocks;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_context_len = max_context_len;
-    p.partition_size = ps;
+    // one partition fits every context: no choice to make
+    p.partition_size = (wl.max_parts > 1) ? ps_hi : ps;
+    p.partition_min = (wl.max_parts > 1 && ps_hi != ps) ? ps : 0;
     p.stages = R;
     p.warps = W;
     p.warp_smem = per_warp;

@@ -42,18 +42,19 @@ def test_status_strings(lib):
 
 
 def test_partition_and_workspace_sizes(lib):
-    # library choice: 16 blocks for small groups, 32 for G >= 4
-    assert lib.paged_attention_partition_size(40, 40, 16, 2048, 0) == 256
-    assert lib.paged_attention_partition_size(64, 8, 16, 32768, 0) == 512
-    assert lib.paged_attention_partition_size(32, 32, 32, 4096, 0) == 512
+    # library choice: a per-call size in [8, 16] blocks (in [16, 32] for G >= 4);
+    # the call reports the lower end, which sizes the workspace
+    assert lib.paged_attention_partition_size(40, 40, 16, 2048, 0) == 128
+    assert lib.paged_attention_partition_size(64, 8, 16, 32768, 0) == 256
+    assert lib.paged_attention_partition_size(32, 32, 32, 4096, 0) == 256
     assert lib.paged_attention_partition_size(32, 32, 16, 4096, 48) == 48
     assert lib.paged_attention_partition_size(32, 32, 16, 4096, 40) == 0      # not a block multiple
     assert lib.paged_attention_partition_size(32, 32, 16, 4096, 1024) == 0    # > 32 blocks
     small = lib.paged_attention_workspace_size(64, 40, 40, 128, 16, 200, 1, 0)
     big = lib.paged_attention_workspace_size(64, 40, 40, 128, 16, 2048, 1, 0)
     assert 0 < small < big
-    # partials: S * parts * H * (D floats + an (m, l) pair)
-    assert big >= 64 * 8 * 40 * (128 * 4 + 8)
+    # partials: S * parts * H * (D floats + an (m, l) pair), parts at the smallest size
+    assert big >= 64 * 16 * 40 * (128 * 4 + 8)
     assert lib.paged_attention_workspace_size(64, 40, 7, 128, 16, 2048, 1, 0) == 0   # G not integral
     assert lib.paged_attention_workspace_size(64, 48, 4, 128, 16, 2048, 1, 0) == 0   # G = 12
     assert lib.paged_attention_workspace_size(64, 40, 40, 96, 16, 2048, 1, 0) == 0   # head_size 96
