@@ -18,7 +18,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -130,54 +129,77 @@ def build_cow_state(device):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of this process's GPU, polled through
+    NVML every 2 ms on a background thread while the timed region runs (it
+    only reads; no setting is changed).  Samples are kept only between
+    mark_start() and mark_end(), i.e. under load."""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, device_index):
+        import threading
+        self.samples, self.max_mhz, self.error = [], None, None
+        self._stop = threading.Event()
+        self._on = threading.Event()
+        self._thread = None
+        self.device_index = device_index
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                return h
+        return pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def _run(self):
+        import pynvml
+        try:
+            h = self._handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = {k: getattr(pynvml, v) for k, v in self.REASONS.items() if hasattr(pynvml, v)}
+            while not self._stop.is_set():
+                if self._on.is_set():
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(mhz), [k for k, m in masks.items() if bits & m]))
+                self._stop.wait(0.002)
+        except Exception as e:              # NVML missing: report no samples
+            self.error = str(e)[:120]
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
+        import threading
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
         return self
 
+    def mark_start(self):
+        self._on.set()
+
+    def mark_end(self):
+        self._on.clear()
+
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(5)
 
     def summary(self):
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                mhz.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not mhz:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml", "error": self.error}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 2 ms polling"}
 
 
 def kernel_source_sha():
@@ -277,6 +299,22 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (ms): every rank takes part in one all-reduce."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(step_bytes, ms_step, world):
+    """Aggregate throughput (GB/s) of `world` replicas each moving step_bytes per step."""
+    return world * step_bytes / (ms_step * 1e-3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -328,28 +366,26 @@ def run_ours(args, rank, world, local_rank):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
-        time.sleep(0.3)
+        time.sleep(0.05)
         torch.cuda.synchronize(device)
+        clk.mark_start()
         start.record(stream)
         for _ in range(args.steps):
             step(record=True)
         end.record(stream)
         torch.cuda.synchronize(device)
+        clk.mark_end()
     if world > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
     dec_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     errors = pkv.read_device_errors()
 
     step_bytes = decode_bytes(lay) + cache_write_bytes(lay)
     if pairs_d is not None:
         step_bytes += 2 * len(pairs) * 2 * Hkv * bs * D * 2
     ms_step = ms_total / args.steps
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_value(step_bytes, ms_step, world)
 
     result = None
     if rank == 0:
@@ -393,48 +429,81 @@ def run_ours(args, rank, world, local_rank):
 
 def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
     """Same step through the C ABI with the step's inputs in pinned host
-    memory: H2D of q, new K/V, slots, tables, lengths (and CoW pairs) and D2H
-    of the output inside the timed region, every step."""
+    memory.  The inputs (q, new K/V, slots, tables, lengths, CoW pairs) sit
+    in one pinned staging buffer and go to the device in one copy; the
+    output comes back in one copy; both are inside the timed region every
+    step.  The step (copy, library calls, copy back) is captured once in a
+    CUDA graph and replayed per step, as a serving loop would; the eager
+    version (one Python call sequence per step) is reported beside it."""
     import torch
     import paged_kv_cache_480_b200 as pkv
-    pin = lambda t: t.detach().cpu().pin_memory()
-    h_q, h_k, h_v = pin(ten["q"]), pin(ten["k_new"]), pin(ten["v_new"])
-    h_sm = torch.from_numpy(lay.slot_mapping).pin_memory()
-    h_bt = torch.from_numpy(lay.block_tables).pin_memory()
-    h_cl = torch.from_numpy(lay.context_lens).pin_memory()
-    h_pairs = torch.from_numpy(np.ascontiguousarray(pairs)).pin_memory() if pairs is not None and len(pairs) else None
-    d = {k: torch.empty_like(v, device=device) for k, v in
-         dict(q=h_q, k=h_k, v=h_v, sm=h_sm, bt=h_bt, cl=h_cl).items()}
-    d_pairs = torch.empty_like(h_pairs, device=device) if h_pairs is not None else None
-    out = torch.empty_like(d["q"])
-    h_out = torch.empty_like(out, device="cpu").pin_memory()
-    stream = torch.cuda.current_stream(device)
+    parts = [("q", ten["q"]), ("k", ten["k_new"]), ("v", ten["v_new"]),
+             ("sm", torch.from_numpy(lay.slot_mapping)), ("bt", torch.from_numpy(lay.block_tables)),
+             ("cl", torch.from_numpy(lay.context_lens))]
+    if pairs is not None and len(pairs):
+        parts.append(("pairs", torch.from_numpy(np.ascontiguousarray(pairs))))
+    offs, total = {}, 0
+    for name, t in parts:
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(total, dtype=torch.uint8, device=device)
+
+    def view(buf, name, t):
+        n = t.numel() * t.element_size()
+        return buf[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+
+    for name, t in parts:
+        view(h_buf, name, t).copy_(t.detach().cpu())
+    d = {name: view(d_buf, name, t) for name, t in parts}
+    out = torch.empty_like(ten["q"])
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     max_ctx = lay.max_context_len
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_sm, h_bt, h_cl))
-    if h_pairs is not None:
-        h2d += h_pairs.numel() * h_pairs.element_size()
+    h2d = sum(t.numel() * t.element_size() for _, t in parts)
     d2h = h_out.numel() * h_out.element_size()
 
-    def step():
-        for k, h in (("q", h_q), ("k", h_k), ("v", h_v), ("sm", h_sm), ("bt", h_bt), ("cl", h_cl)):
-            d[k].copy_(h, non_blocking=True)
-        if h_pairs is not None:
-            d_pairs.copy_(h_pairs, non_blocking=True)
-            pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], d_pairs, stream=stream)
+    def body(stream):
+        d_buf.copy_(h_buf, non_blocking=True)
+        if "pairs" in d:
+            pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], d["pairs"], stream=stream)
         pkv.reshape_and_cache(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], stream=stream)
         pkv.paged_attention_decode(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"],
                                    lay.scale, max_context_len=max_ctx, workspace=ws, stream=stream)
         h_out.copy_(out, non_blocking=True)
-        stream.synchronize()
 
-    for _ in range(3):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    return {"value": step_bytes / dt / 1e9, "unit": "GB/s", "us_per_step": dt * 1e6,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    def timed(run, sync):
+        for _ in range(3):
+            run()
+            sync()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            run()
+            sync()
+        return (time.perf_counter() - t0) / args.steps
+
+    stream = torch.cuda.current_stream(device)
+    eager = timed(lambda: body(stream), stream.synchronize)
+    result = {"value": step_bytes / eager / 1e9, "unit": "GB/s", "us_per_step": eager * 1e6,
+              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager"}
+    try:
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            body(cap)                       # warm the capture stream
+            cap.synchronize()
+            with torch.cuda.graph(graph, stream=cap):
+                body(cap)
+        stream.wait_stream(cap)
+        replay = timed(graph.replay, torch.cuda.synchronize)
+        assert pkv.read_device_errors() == 0
+        result.update({"value": step_bytes / replay / 1e9, "us_per_step": replay * 1e6,
+                       "mode": "cuda graph of the step, replayed per step",
+                       "eager_value": step_bytes / eager / 1e9, "eager_us_per_step": eager * 1e6})
+        del graph
+    except Exception as e:                  # capture unavailable: keep the eager number
+        result["graph_error"] = str(e)[:200]
+    return result
 
 
 def main():
