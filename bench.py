@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="cache write fused into the decode (paged_attention_decode_append)")
     return ap.parse_args()
 
 
@@ -338,21 +340,29 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(device)
     nparts = pkv.paged_attention_partition_size(H, Hkv, bs, max_ctx, ps)
     split = max_ctx > nparts
-    launches_per_step = 2 + (1 if split else 0) + (1 if pairs_d is not None else 0)
+    launches_per_step = (1 if args.fused else 2) + (1 if split else 0) + (1 if pairs_d is not None else 0)
 
     ev = []
 
     def step(record=False):
         if pairs_d is not None:
             pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], pairs_d, stream=stream)
-        pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm, stream=stream)
+        if not args.fused:
+            pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm,
+                                  stream=stream)
         if record:
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-        pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
-                                   max_context_len=max_ctx, partition_size=ps, workspace=ws,
-                                   stream=stream)
+        if args.fused:
+            pkv.paged_attention_decode_append(out, ten["q"], ten["k_new"], ten["v_new"], ten["k_cache"],
+                                              ten["v_cache"], sm, bt, cl, lay.scale,
+                                              max_context_len=max_ctx, partition_size=ps,
+                                              workspace=ws, stream=stream)
+        else:
+            pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                                       max_context_len=max_ctx, partition_size=ps, workspace=ws,
+                                       stream=stream)
         if record:
             b.record(stream)
             ev.append((a, b))
@@ -392,7 +402,9 @@ def run_ours(args, rank, world, local_rank):
         peak, peak_kind = peaks()
         dec_avg = sum(dec_ms) / len(dec_ms)
         achieved = decode_bytes(lay) / (dec_avg * 1e-3) / 1e9
-        roof = {"kernel": "paged_attention_decode (decode" + (" + lse merge)" if split else ")"),
+        kname = "paged_attention_decode_append (fused cache write + decode" if args.fused else \
+            "paged_attention_decode (decode"
+        roof = {"kernel": kname + (" + lse merge)" if split else ")"),
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind,
                 "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
@@ -410,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
                              "mean_context_len": float(lay.context_lens.mean()),
                              "partition_size": nparts, "split_context": split,
                              "cow_pairs": 0 if pairs is None else int(len(pairs)),
-                             "step_bytes": step_bytes,
+                             "step_bytes": step_bytes, "fused_cache_write": bool(args.fused),
                              "l2": f"inputs larger than L2: {lay.kv_bytes() / 1e9:.2f} GB of K/V per step",
                              "parallelism": f"replicas x{world}"},
                   "roofline": roof, "gpu_launches": launches_per_step * args.steps,
@@ -466,25 +478,37 @@ def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
         d_buf.copy_(h_buf, non_blocking=True)
         if "pairs" in d:
             pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], d["pairs"], stream=stream)
-        pkv.reshape_and_cache(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], stream=stream)
-        pkv.paged_attention_decode(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"],
-                                   lay.scale, max_context_len=max_ctx, workspace=ws, stream=stream)
+        if args.fused:
+            pkv.paged_attention_decode_append(out, d["q"], d["k"], d["v"], ten["k_cache"], ten["v_cache"],
+                                              d["sm"], d["bt"], d["cl"], lay.scale,
+                                              max_context_len=max_ctx, workspace=ws, stream=stream)
+        else:
+            pkv.reshape_and_cache(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], stream=stream)
+            pkv.paged_attention_decode(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"],
+                                       lay.scale, max_context_len=max_ctx, workspace=ws, stream=stream)
         h_out.copy_(out, non_blocking=True)
 
+    n_steps = max(args.steps, 200)
+
     def timed(run, sync):
+        """Median wall time of one step (host sync every step; the median
+        keeps host scheduling jitter out of a ~0.3 ms step)."""
         for _ in range(3):
             run()
             sync()
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
+        times = []
+        for _ in range(n_steps):
+            t0 = time.perf_counter()
             run()
             sync()
-        return (time.perf_counter() - t0) / args.steps
+            times.append(time.perf_counter() - t0)
+        return statistics.median(times)
 
     stream = torch.cuda.current_stream(device)
     eager = timed(lambda: body(stream), stream.synchronize)
     result = {"value": step_bytes / eager / 1e9, "unit": "GB/s", "us_per_step": eager * 1e6,
-              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager"}
+              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager",
+              "timing": f"median of {n_steps} wall-clock steps, each ending in a host sync"}
     try:
         cap = torch.cuda.Stream(device)
         cap.wait_stream(stream)

@@ -126,6 +126,35 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                                   pkv_dtype dtype, int partition_size, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * paged_attention_decode_append -- reshape_and_cache of one new token per
+ * sequence fused into paged_attention_decode (one launch fewer per step).
+ *
+ * Defines exactly what reshape_and_cache(key, value, ..., slot_mapping)
+ * followed by paged_attention_decode(...) defines: the decode step appends
+ * the new token's key/value ("PyTorch-CUDA-v2.9 image enables
+ * PagedAttention", PagedAttention section) and attends over the context
+ * including it.  Token s's rows key[s][g] / value[s][g] (token stride in
+ * elements, multiple of 16 bytes) go to slot slot_mapping[s] (int64,
+ * device); a negative slot means no new token for that sequence.  The slot
+ * must be the slot of position context_lens[s] - 1 (the block-table entry of
+ * that position and its offset); otherwise nothing is written for that
+ * sequence and PKV_DEVERR_SLOT is set.  The block holding the slot must not
+ * be shared with another sequence (copy_blocks first, as for
+ * reshape_and_cache).  Every other argument, the workspace and the errors
+ * are those of paged_attention_decode.
+ * ------------------------------------------------------------------------- */
+pkv_status paged_attention_decode_append(void* out, const void* q, const void* key,
+                                         const void* value, void* k_cache, void* v_cache,
+                                         const int64_t* slot_mapping, const int32_t* block_tables,
+                                         const int32_t* context_lens, float scale,
+                                         int num_kv_heads, int block_size, int num_seqs,
+                                         int num_heads, int head_size, int num_blocks,
+                                         int max_blocks_per_seq, int max_context_len,
+                                         int64_t key_token_stride, int64_t value_token_stride,
+                                         pkv_dtype dtype, int partition_size, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace paged_attention_decode needs for these sizes (0 on bad
  * arguments).  partition_size as in paged_attention_decode. */
 size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

@@ -60,6 +60,9 @@ def load_library(path=LIB_PATH):
         lib.reshape_and_cache.restype = I
         lib.copy_blocks.argtypes = [P, P, I, P, I, I, I64, P]
         lib.copy_blocks.restype = I
+        lib.paged_attention_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I,
+                                                      I64, I64, I, I, P, SZ, P]
+        lib.paged_attention_decode_append.restype = I
         lib.paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P]
         lib.paged_attention_decode_noalloc.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
@@ -196,6 +199,50 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream, q.device))
     _check(st, "paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping,
+                                  block_tables, context_lens, scale, max_context_len=None,
+                                  partition_size=0, workspace=None, stream=None):
+    """reshape_and_cache of one new token per sequence fused into the decode
+    (paged_attention_decode_append in pagedkv.h).  key/value: [S, Hkv, D]
+    (token stride may exceed Hkv * D); slot_mapping: int64 [S], each the slot
+    of position context_lens[s] - 1, or negative for none."""
+    import torch
+    lib = load_library()
+    S, H, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if tuple(key.shape) != (S, Hkv, D) or tuple(value.shape) != (S, Hkv, D):
+        raise ValueError("key/value must be [num_seqs, num_kv_heads, head_size]")
+    if key.stride(2) != 1 or key.stride(1) != D or value.stride(2) != 1 or value.stride(1) != D:
+        raise ValueError("key/value heads must be contiguous within a token")
+    for t in (key, value, k_cache, v_cache, out):
+        if t.dtype != q.dtype:
+            raise ValueError("all tensors must share q's dtype")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != S:
+        raise TypeError("slot_mapping must be int64 [num_seqs]")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    MB = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = MB * bs
+    code = _dtype_code(q)
+    need = lib.paged_attention_workspace_size(S, H, Hkv, D, bs, max_context_len, code, partition_size)
+    if need == 0:
+        raise PagedKVError(2, "paged_attention_workspace_size")
+    if workspace is None:
+        workspace = default_workspace(q.device, need)
+    st = lib.paged_attention_decode_append(
+        _contig(out, "out"), _contig(q, "q"), _cuda(key, "key"), _cuda(value, "value"),
+        _contig(k_cache, "k_cache"), _contig(v_cache, "v_cache"), _contig(slot_mapping, "slot_mapping"),
+        _contig(block_tables, "block_tables"), _contig(context_lens, "context_lens"), float(scale),
+        Hkv, bs, S, H, D, NB, MB, int(max_context_len), key.stride(0), value.stride(0), code,
+        int(partition_size), _cuda(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+    _check(st, "paged_attention_decode_append")
     return out
 
 

@@ -51,6 +51,13 @@ struct DecodeParams {
     int num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int partition_size;     // PS tokens, a multiple of block_size, <= 32 blocks
     int partition_min;      // > 0: choose PS in [partition_min, partition_size] on the device
+    // Fused cache write (all null for a plain decode): the step's new token
+    // of sequence s, rows key[s][g] / value[s][g], goes to slot
+    // slot_mapping[s], which must be the slot of position context_len - 1.
+    const void* key;
+    const void* value;
+    const int64_t* slot_mapping;
+    int64_t key_stride, value_stride;   // elements between sequences
     int stages;             // R
     int warps;              // W consumer warps per CTA
     uint32_t warp_smem;     // bytes of one warp's region
@@ -70,7 +77,9 @@ struct StageMeta {
     int nvalid;  // valid tokens in this block (0 = nothing to read)
     int flags;   // kFirst | kLast | kWhole
     int qslot;
-    int pad;
+    int newrow;  // row of this block that takes the step's new token, or -1
+    int64_t slot;
+    int64_t pad;
 };
 constexpr int kFirst = 1, kLast = 2, kWhole = 4;
 
@@ -80,8 +89,12 @@ struct WarpSmem {
     using S = DecodeShape<T, D, BS, G>;
     __host__ __device__ static constexpr uint32_t ring(int) { return 0; }
     __host__ __device__ static constexpr uint32_t qbuf(int R) { return (uint32_t)R * 2 * S::TILE; }
-    __host__ __device__ static constexpr uint32_t meta(int R) {
+    // new-token K and V rows of each stage (fused cache write)
+    __host__ __device__ static constexpr uint32_t nbuf(int R) {
         return qbuf(R) + (uint32_t)R * S::QBYTES;
+    }
+    __host__ __device__ static constexpr uint32_t meta(int R) {
+        return nbuf(R) + (uint32_t)R * 2 * S::ROW;
     }
     __host__ __device__ static constexpr uint32_t bars(int R) {
         return meta(R) + (uint32_t)R * sizeof(StageMeta);
@@ -99,6 +112,7 @@ struct Item {
     int nblk;     // stages the item occupies (>= 1)
     int whole;    // the item is the whole sequence
     int tbl;      // lane j holds the item's j-th physical block id
+    int64_t slot; // fused cache write: slot of the new token if this item holds it, else -1
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -526,6 +540,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
     unsigned char* wb = smem + p.seq_smem + (size_t)warp * p.warp_smem;
     unsigned char* ring = wb + L::ring(R);
     unsigned char* qbuf = wb + L::qbuf(R);
+    unsigned char* nbuf = wb + L::nbuf(R);
     StageMeta* meta = reinterpret_cast<StageMeta*>(wb + L::meta(R));
     const uint32_t bar0 = smem_addr(wb + L::bars(R));
     int PS = p.partition_size;
@@ -577,6 +592,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         it.idx = idx;
         it.s = it.g = it.part = it.tok0 = it.ntok = it.whole = it.tbl = 0;
         it.nblk = 0;
+        it.slot = -1;
         if (idx >= n_items) return it;
         const int jsp = idx / Hkv;
         it.g = idx - jsp * Hkv;
@@ -594,6 +610,8 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         it.nblk = max(used, 1);
         if (lane < used)
             it.tbl = __ldg(p.block_tables + (size_t)lo * p.max_blocks_per_seq + it.tok0 / BS + lane);
+        if (p.slot_mapping != nullptr && it.ntok > 0 && it.tok0 + it.ntok == s_len[lo])
+            it.slot = __ldg(p.slot_mapping + lo);
         return it;
     };
     auto next_index = [&]() -> int {
@@ -624,17 +642,34 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         const bool bad = nvalid > 0 && (phys < 0 || phys >= p.num_blocks);
         if (bad) nvalid = 0;
         const bool first = pj == 0, last = pj == P.nblk - 1;
+        // Fused cache write: the last block of the item that ends the sequence
+        // holds the new token at row newrow; its slot must be that position.
+        int newrow = -1;
+        if (last && P.slot >= 0 && nvalid > 0) {
+            newrow = nvalid - 1;
+            if (P.slot != (int64_t)phys * BS + newrow) newrow = -2;   // not the last position
+        }
         if (lane == 0) {
             StageMeta m;
             m.item = P.idx; m.s = P.s; m.g = P.g; m.part = P.part;
             m.nvalid = nvalid;
             m.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (P.whole ? kWhole : 0);
             m.qslot = qslot_ctr;
+            m.newrow = newrow < 0 ? -1 : newrow;
+            m.slot = P.slot;
             m.pad = 0;
             meta[st] = m;
             const uint32_t bar = bar0 + 8 * st;
-            const uint32_t bytes = (first ? S::QBYTES : 0) + (nvalid > 0 ? 2 * S::TILE : 0);
+            const uint32_t bytes = (first ? S::QBYTES : 0) + (nvalid > 0 ? 2 * S::TILE : 0) +
+                                   (newrow >= 0 ? 2 * S::ROW : 0);
             mbar_arrive_expect_tx(bar, bytes);
+            if (newrow >= 0) {
+                const T* kn = reinterpret_cast<const T*>(p.key) + (size_t)P.s * p.key_stride + (size_t)P.g * D;
+                const T* vn = reinterpret_cast<const T*>(p.value) + (size_t)P.s * p.value_stride + (size_t)P.g * D;
+                bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW), kn, S::ROW, bar);
+                bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW + S::ROW), vn, S::ROW, bar);
+            }
+            if (newrow == -2) flag_error(p.errors, PKV_DEVERR_SLOT);
             if (first)
                 bulk_g2s(smem_addr(qbuf + qslot_ctr * S::QBYTES),
                          qg + ((size_t)P.s * p.num_heads + (size_t)P.g * G) * D, S::QBYTES, bar);
@@ -676,6 +711,24 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         }
         const StageMeta mt = meta[cons_st];
         if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, p.scale_log2);
+        if (mt.newrow >= 0) {
+            // Fused cache write: put the new token's K and V rows into the tile
+            // (it holds the slot's old bytes) and into the cache slot.
+            unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
+            const unsigned char* nb = nbuf + (size_t)cons_st * 2 * S::ROW;
+            const size_t slot_off = (size_t)mt.slot / BS * Hkv * tile_elems +
+                                    (size_t)mt.g * tile_elems + (size_t)(mt.slot % BS) * D;
+            for (int ch = lane; ch < 2 * S::ROW / 16; ch += 32) {
+                const int v = ch >= S::ROW / 16;
+                const int c16 = ch - v * (S::ROW / 16);
+                const uint4 w = reinterpret_cast<const uint4*>(nb + v * S::ROW)[c16];
+                reinterpret_cast<uint4*>(Kt + v * S::TILE + mt.newrow * S::ROW)[c16] = w;
+                T* cache = const_cast<T*>(v ? vc : kc);
+                reinterpret_cast<uint4*>(cache + slot_off)[c16] = w;
+            }
+            fence_proxy_async();     // these generic writes precede the stage's next bulk copy
+            __syncwarp();
+        }
         if (mt.nvalid > 0) {
             const unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
             cons.block(Kt, Kt + S::TILE, mt.nvalid, p.scale_log2);

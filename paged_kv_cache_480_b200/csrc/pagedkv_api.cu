@@ -162,13 +162,24 @@ pkv_status paged_attention_workspace_init(void* workspace, size_t workspace_byte
     return PKV_OK;
 }
 
-pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
-                                  const void* v_cache, const int32_t* block_tables,
-                                  const int32_t* context_lens, float scale, int num_kv_heads,
-                                  int block_size, int num_seqs, int num_heads, int head_size,
-                                  int num_blocks, int max_blocks_per_seq, int max_context_len,
-                                  pkv_dtype dtype, int partition_size, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused cache write of paged_attention_decode_append (null: none).
+struct AppendArgs {
+    const void* key;
+    const void* value;
+    const int64_t* slot_mapping;
+    int64_t key_stride, value_stride;
+};
+
+pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens, float scale,
+                       int num_kv_heads, int block_size, int num_seqs, int num_heads,
+                       int head_size, int num_blocks, int max_blocks_per_seq, int max_context_len,
+                       pkv_dtype dtype, int partition_size, void* workspace,
+                       size_t workspace_bytes, void* stream, const AppendArgs* app) {
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return PKV_ERR_INVALID_ARG;
     pkv_status st = check_shape(num_seqs, num_heads, num_kv_heads, head_size, block_size,
@@ -233,6 +244,13 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
     // one partition fits every context: no choice to make
     p.partition_size = (wl.max_parts > 1) ? ps_hi : ps;
     p.partition_min = (wl.max_parts > 1 && ps_hi != ps) ? ps : 0;
+    if (app) {
+        p.key = app->key;
+        p.value = app->value;
+        p.slot_mapping = app->slot_mapping;
+        p.key_stride = app->key_stride;
+        p.value_stride = app->value_stride;
+    }
     p.stages = R;
     p.warps = W;
     p.warp_smem = per_warp;
@@ -268,6 +286,48 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
         if (e != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int num_kv_heads,
+                                  int block_size, int num_seqs, int num_heads, int head_size,
+                                  int num_blocks, int max_blocks_per_seq, int max_context_len,
+                                  pkv_dtype dtype, int partition_size, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                       block_size, num_seqs, num_heads, head_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, dtype, partition_size, workspace, workspace_bytes, stream,
+                       nullptr);
+}
+
+pkv_status paged_attention_decode_append(void* out, const void* q, const void* key,
+                                         const void* value, void* k_cache, void* v_cache,
+                                         const int64_t* slot_mapping, const int32_t* block_tables,
+                                         const int32_t* context_lens, float scale,
+                                         int num_kv_heads, int block_size, int num_seqs,
+                                         int num_heads, int head_size, int num_blocks,
+                                         int max_blocks_per_seq, int max_context_len,
+                                         int64_t key_token_stride, int64_t value_token_stride,
+                                         pkv_dtype dtype, int partition_size, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+    if (!key || !value || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    const int64_t eb = elem_bytes(dtype);
+    if (key_token_stride < (int64_t)num_kv_heads * head_size ||
+        value_token_stride < (int64_t)num_kv_heads * head_size ||
+        (key_token_stride * eb) % 16 || (value_token_stride * eb) % 16)
+        return PKV_ERR_INVALID_ARG;
+    const AppendArgs app{key, value, slot_mapping, key_token_stride, value_token_stride};
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                       block_size, num_seqs, num_heads, head_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, dtype, partition_size, workspace, workspace_bytes, stream,
+                       &app);
 }
 
 pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
