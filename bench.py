@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap"],
+                    help="swap: swap_blocks between the GPU pool and a pinned host pool")
     ap.add_argument("--fused", action="store_true",
                     help="cache write fused into the decode (paged_attention_decode_append)")
     return ap.parse_args()
@@ -530,6 +532,64 @@ def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
     return result
 
 
+def run_swap(args, rank, world, local_rank):
+    """swap_blocks throughput, device <-> pinned host, against a contiguous
+    pinned copy of the same size measured in the same run (the host link's
+    ceiling).  Pools shaped like the OPT-13B layer (40 heads x 16 x 128 fp16 =
+    160 KB per block per cache), K and V, 512 scattered blocks each way."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    shape = (40, 16, 128)
+    NBd, NBh, n = 2048, 1024, 512
+    kd = torch.randn((NBd,) + shape, device=device).half()
+    vd = torch.randn((NBd,) + shape, device=device).half()
+    kh = torch.empty((NBh,) + shape, dtype=torch.float16).pin_memory()
+    vh = torch.empty_like(kh).pin_memory()
+    rng = np.random.default_rng(480)
+    out_map = torch.from_numpy(np.stack([rng.choice(NBd, n, replace=False),
+                                         rng.choice(NBh, n, replace=False)], 1).astype(np.int64)).to(device)
+    in_map = torch.from_numpy(np.stack([rng.choice(NBh, n, replace=False),
+                                        rng.choice(NBd, n, replace=False)], 1).astype(np.int64)).to(device)
+    nbytes = 2 * n * kd[0].numel() * 2
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b) / args.steps * 1e-3
+
+    t_out = timed(lambda: pkv.swap_blocks([kd, vd], [kh, vh], out_map, stream=stream))
+    t_in = timed(lambda: pkv.swap_blocks([kh, vh], [kd, vd], in_map, stream=stream))
+    big_h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    big_d = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    t_h2d = timed(lambda: big_d.copy_(big_h, non_blocking=True))
+    t_d2h = timed(lambda: big_h.copy_(big_d, non_blocking=True))
+    assert pkv.read_device_errors() == 0
+    res = []
+    for name, t, tp in (("device->host", t_out, t_d2h), ("host->device", t_in, t_h2d)):
+        ach, peak = nbytes / t / 1e9, nbytes / tp / 1e9
+        res.append({"metric": f"swap_blocks {name} GB/s", "value": ach, "unit": "GB/s", "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+                    "data": "synthetic",
+                    "config": {"workload": "swap 512 scattered blocks x (K, V) of 160 KB", "bytes": nbytes},
+                    "roofline": {"bound": "host link", "achieved": ach, "peak": peak, "unit": "GB/s",
+                                 "frac": ach / peak,
+                                 "peak_kind": "contiguous pinned copy of the same bytes, this run"},
+                    "gpu_launches": args.steps})
+    return res
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -548,6 +608,11 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.measure == "swap":
+            for line in run_swap(args, rank, world, local_rank):
+                if rank == 0:
+                    print(json.dumps(line), flush=True)
+            return
         res = run_ours(args, rank, world, local_rank)
         if res is not None:
             print(json.dumps(res), flush=True)

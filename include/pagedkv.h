@@ -253,6 +253,30 @@ pkv_status paged_attention_decode_noalloc(void* out, const void* q, const void* 
                                           int max_blocks_per_seq, int max_context_len,
                                           pkv_dtype dtype, int partition_size, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * swap_blocks -- block copy between two pools, typically the GPU pool and a
+ * pinned host pool ("Efficient Memory Management for Large Language Model
+ * Serving with PagedAttention" summary page, section 2: the KV-cache manager
+ * keeps a block pool in GPU memory and one in CPU memory for swapping; the
+ * scheduler recovers preempted requests by swapping).
+ *
+ * Defines: for every cache c < num_caches and pair i, block
+ * block_mapping[i][1] of dst_caches[c] becomes a bit copy of block
+ * block_mapping[i][0] of src_caches[c] (block_bytes bytes each).
+ *   src_caches, dst_caches  HOST arrays of num_caches pointers (e.g. the K
+ *                  and V caches of every layer, <= 512); each pointer is
+ *                  device memory or pinned (page-locked, mapped) host memory,
+ *                  checked on the host (PKV_ERR_INVALID_ARG otherwise)
+ *   block_mapping  int64 [num_pairs][2] (src, dst) in device or pinned host
+ *                  memory; ids outside [0, src_num_blocks) / [0,
+ *                  dst_num_blocks) are skipped and flag PKV_DEVERR_COPY_ID
+ * Destinations must be distinct.  Asynchronous on the stream; the host pool
+ * must stay alive until the stream has passed the copy.
+ * ------------------------------------------------------------------------- */
+pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, int num_caches,
+                       const int64_t* block_mapping, int num_pairs, int src_num_blocks,
+                       int dst_num_blocks, int64_t block_bytes, void* stream);
+
 /* Synchronise the stream, return the sticky device-check bits of the
  * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
  * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */
@@ -290,6 +314,16 @@ pkv_status pkv_bm_append_slot(pkv_block_manager* bm, int64_t seq_id, int64_t* sl
  * status; *num_done tells how many sequences were served. */
 pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, int n,
                                int64_t* slots, int64_t* cow_pairs, int* num_cow, int* num_done);
+/* Swap a whole sequence from manager bm to manager host (e.g. GPU pool to
+ * host pool; the reverse call swaps it back in), all or nothing: host gets
+ * the sequence with fresh private blocks (sharing ends at a swap), bm drops
+ * its references.  pairs[2 * j], pairs[2 * j + 1] = (block in bm, block in
+ * host) for the j-th logical block, the copies to pass to swap_blocks;
+ * *num_pairs = the sequence's block count.  PKV_ERR_OUT_OF_BLOCKS (nothing
+ * changed) if host has too few free blocks; PKV_ERR_INVALID_ARG if capacity
+ * is too small or the block sizes differ. */
+pkv_status pkv_bm_swap_out(pkv_block_manager* bm, pkv_block_manager* host, int64_t seq_id,
+                           int64_t* pairs, int capacity, int* num_pairs);
 pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
 /* Copy the sequence's table into out[0 .. capacity); *num_blocks = its length. */
 pkv_status pkv_bm_block_table(const pkv_block_manager* bm, int64_t seq_id, int32_t* out,

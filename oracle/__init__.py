@@ -44,6 +44,7 @@ def _load():
         lib.orc_lse_merge.argtypes = [P, P, P, P, I64, I, I]
         lib.orc_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I64, I64]
         lib.orc_copy_blocks.argtypes = [P, I, P, I, I64]
+        lib.orc_swap_blocks.argtypes = [P, P, I, P, I, I64]
         lib.orc_round.argtypes = [P, P, I, I64]
         lib.orc_load.argtypes = [P, I, I64]
         lib.orc_load.restype = D
@@ -190,3 +191,17 @@ def copy_blocks(caches, block_mapping):
         assert c.flags.c_contiguous and c[0].nbytes == block_bytes
     arr = (ctypes.c_void_p * len(caches))(*[c.ctypes.data for c in caches])
     _load().orc_copy_blocks(arr, len(caches), _ptr(bm), bm.shape[0], block_bytes)
+
+
+def swap_blocks(src_pools, dst_pools, block_mapping):
+    """dst_pools[c][dst] = src_pools[c][src] for every (src, dst) pair, in place."""
+    bm = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    if len(src_pools) == 0 or bm.shape[0] == 0:
+        return
+    block_bytes = src_pools[0][0].nbytes
+    for a in list(src_pools) + list(dst_pools):
+        assert a.flags.c_contiguous and a[0].nbytes == block_bytes
+    n = len(src_pools)
+    sa = (ctypes.c_void_p * n)(*[a.ctypes.data for a in src_pools])
+    da = (ctypes.c_void_p * n)(*[a.ctypes.data for a in dst_pools])
+    _load().orc_swap_blocks(sa, da, n, _ptr(bm), bm.shape[0], block_bytes)

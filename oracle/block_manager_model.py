@@ -104,6 +104,26 @@ class BlockManagerModel:
         self.lens[seq] = t + 1
         return b * self.block_size + off, cow
 
+    def swap_out(self, seq, host):
+        """Move the whole sequence to the host-pool manager `host`, all or
+        nothing; returns the (device block, host block) copies to make.  The
+        host copies are private to the sequence (sharing ends at a swap)."""
+        table = self.tables[seq]
+        if len(table) > len(host.free):
+            raise OutOfBlocks(len(table))
+        dst = host._take(len(table))
+        for d, b in zip(dst, table):
+            host.fill[d] = self.fill[b]
+        host.tables[seq] = list(dst)
+        host.lens[seq] = self.lens[seq]
+        pairs = list(zip(table, dst))
+        self.free_seq(seq)
+        return pairs
+
+    def swap_in(self, seq, host):
+        """The reverse of swap_out: the sequence returns from `host`."""
+        return host.swap_out(seq, self)
+
     def free_seq(self, seq):
         for b in self.tables.pop(seq):
             self._release(b)

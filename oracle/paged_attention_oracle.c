@@ -338,3 +338,17 @@ void orc_copy_blocks(void** caches, int num_layers, const int64_t* block_mapping
                    (const char*)caches[layer] + src * block_bytes, (size_t)block_bytes);
         }
 }
+
+/* ---------------------------------------------------------------------------
+ * Swap between two block pools [P5 s.2: a block pool in GPU memory and one
+ * in CPU memory, the latter for swapping; recovery by swap]: for every cache
+ * c and pair i, block dst of dst_pools[c] becomes a copy of block src of
+ * src_pools[c].  Pairs are applied in order.
+ * ------------------------------------------------------------------- */
+void orc_swap_blocks(void** src_pools, void** dst_pools, int num_caches, const int64_t* mapping,
+                     int num_pairs, int64_t block_bytes) {
+    for (int c = 0; c < num_caches; ++c)
+        for (int i = 0; i < num_pairs; ++i)
+            memcpy((char*)dst_pools[c] + mapping[2 * i + 1] * block_bytes,
+                   (const char*)src_pools[c] + mapping[2 * i] * block_bytes, (size_t)block_bytes);
+}

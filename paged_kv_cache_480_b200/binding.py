@@ -65,6 +65,10 @@ def load_library(path=LIB_PATH):
         lib.paged_attention_decode_append.restype = I
         lib.paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P]
         lib.paged_attention_decode_noalloc.restype = I
+        lib.swap_blocks.argtypes = [P, P, I, P, I, I, I, I64, P]
+        lib.swap_blocks.restype = I
+        lib.pkv_bm_swap_out.argtypes = [P, P, I64, P, I, ctypes.POINTER(I)]
+        lib.pkv_bm_swap_out.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         lib.pkv_read_device_errors.restype = I
         lib.pkv_bm_create.argtypes = [I, I, P, ctypes.POINTER(P)]
@@ -320,6 +324,31 @@ def copy_blocks(k_caches, v_caches, block_mapping, stream=None):
     _check(st, "copy_blocks")
 
 
+def swap_blocks(src_caches, dst_caches, block_mapping, stream=None):
+    """Block copies between two pools (device or pinned host memory), e.g. the
+    K and V caches of every layer: dst_caches[c][dst] = src_caches[c][src]
+    for each (src, dst) row of block_mapping (int64 [N, 2], device or pinned)."""
+    import torch
+    lib = load_library()
+    if len(src_caches) != len(dst_caches) or not src_caches:
+        raise ValueError("need matching non-empty lists of caches")
+    if block_mapping.dtype != torch.int64:
+        raise TypeError("block_mapping must be int64")
+    block_bytes = src_caches[0][0].numel() * src_caches[0].element_size()
+    for c in list(src_caches) + list(dst_caches):
+        if c[0].numel() * c.element_size() != block_bytes or not c.is_contiguous():
+            raise ValueError("all pools must be contiguous with equal block sizes")
+    n = len(src_caches)
+    sarr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in src_caches])
+    darr = (ctypes.c_void_p * n)(*[c.data_ptr() for c in dst_caches])
+    dev = next((c.device for c in list(src_caches) + list(dst_caches) if c.is_cuda), None)
+    s = _stream(stream, dev) if dev is not None else ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.swap_blocks(sarr, darr, n, ctypes.c_void_p(block_mapping.data_ptr()),
+                         block_mapping.numel() // 2, src_caches[0].shape[0], dst_caches[0].shape[0],
+                         block_bytes, s)
+    _check(st, "swap_blocks")
+
+
 def read_device_errors(stream=None):
     """Synchronise the stream and return (and clear) the sticky device-check bits."""
     import torch
@@ -387,6 +416,18 @@ class BlockManager:
 
     def free(self, seq):
         _check(self._lib.pkv_bm_free(self._h, seq), "pkv_bm_free")
+
+    def swap_out(self, host, seq):
+        """Move sequence seq to manager `host` (all or nothing); returns int64
+        [n, 2] (block here, block in host) pairs for swap_blocks.  Swapping
+        back in is host.swap_out(self, seq)."""
+        import numpy as np
+        cap = max(self.num_blocks, host.num_blocks)
+        pairs = np.empty((cap, 2), np.int64)
+        n = ctypes.c_int()
+        st = self._lib.pkv_bm_swap_out(self._h, host._h, seq, pairs.ctypes.data, cap, ctypes.byref(n))
+        _check(st, "pkv_bm_swap_out")
+        return pairs[:n.value].copy()
 
     def block_table(self, seq):
         import numpy as np

@@ -156,6 +156,34 @@ pkv_status pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, in
     return PKV_OK;
 }
 
+pkv_status pkv_bm_swap_out(pkv_block_manager* bm, pkv_block_manager* host, int64_t seq_id,
+                           int64_t* pairs, int capacity, int* num_pairs) {
+    if (!bm || !host || bm == host || !num_pairs || capacity < 0 || (capacity > 0 && !pairs))
+        return PKV_ERR_INVALID_ARG;
+    if (bm->block_size != host->block_size) return PKV_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end() || host->seqs.count(seq_id)) return PKV_ERR_NOT_FOUND;
+    const std::vector<int32_t>& table = it->second.table;
+    const int n = (int)table.size();
+    *num_pairs = n;
+    if (n > capacity) return PKV_ERR_INVALID_ARG;
+    if ((size_t)n > host->free_list.size()) return PKV_ERR_OUT_OF_BLOCKS;   // nothing changed
+    pkv_block_manager::Seq hs;
+    hs.len = it->second.len;
+    hs.table.reserve(n);
+    for (int j = 0; j < n; ++j) {
+        const int32_t d = host->take();
+        host->fill[d] = bm->fill[table[j]];
+        hs.table.push_back(d);
+        pairs[2 * j] = table[j];
+        pairs[2 * j + 1] = d;
+    }
+    host->seqs.emplace(seq_id, std::move(hs));
+    for (int32_t b : table) bm->release(b);
+    bm->seqs.erase(it);
+    return PKV_OK;
+}
+
 pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
     if (!bm) return PKV_ERR_INVALID_ARG;
     auto it = bm->seqs.find(seq_id);

@@ -72,6 +72,43 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyBlocksParams
     for (; i < n; i += blockDim.x) d[i] = s[i];
 }
 
+// Swap between a device pool and a pinned host pool (either direction): the
+// host side is read or written in place through unified addressing, so a
+// swap of scattered blocks is one launch.  grid = (pairs, caches); each CTA
+// moves one block with 16-byte vectors, eight loads in flight per thread to
+// cover the host link's latency.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const SwapBlocksParams p) {
+    griddep_wait();
+    griddep_launch();
+    const int pair = blockIdx.x, c = blockIdx.y;
+    const int64_t src = p.block_mapping[2 * (int64_t)pair];
+    const int64_t dst = p.block_mapping[2 * (int64_t)pair + 1];
+    if (src < 0 || src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
+        if (threadIdx.x == 0 && c == 0) flag_error(p.errors, PKV_DEVERR_COPY_ID);
+        return;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(p.src[c]) +
+                                                    src * p.block_bytes);
+    uint4* d = reinterpret_cast<uint4*>(static_cast<unsigned char*>(p.dst[c]) + dst * p.block_bytes);
+    const int64_t n = p.block_bytes / 16;
+    int64_t i = threadIdx.x;
+    constexpr int U = 8;
+    for (; i + (U - 1) * (int64_t)blockDim.x < n; i += U * (int64_t)blockDim.x) {
+        uint4 v[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) v[k] = s[i + k * blockDim.x];
+#pragma unroll
+        for (int k = 0; k < U; ++k) d[i + k * blockDim.x] = v[k];
+    }
+    for (; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+cudaError_t launch_swap_blocks(const SwapBlocksParams& p, int num_pairs, int num_caches,
+                               cudaStream_t stream) {
+    if (num_pairs == 0 || num_caches == 0) return cudaSuccess;
+    return launch_pdl(swap_blocks_kernel, dim3(num_pairs, num_caches), dim3(256), 0, stream, p);
+}
+
 cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cudaStream_t stream) {
     const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.row_bytes / 16);
     if (total == 0) return cudaSuccess;

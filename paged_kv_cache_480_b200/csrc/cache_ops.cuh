@@ -30,6 +30,18 @@ struct CopyBlocksParams {
     int64_t num_blocks;
 };
 
+struct SwapBlocksParams {
+    const void* src[2 * kMaxLayers];
+    void* dst[2 * kMaxLayers];
+    const int64_t* block_mapping;   // [pairs][2] (src, dst), device-accessible
+    unsigned int* errors;
+    int64_t block_bytes;
+    int64_t src_blocks, dst_blocks;
+};
+
+cudaError_t launch_swap_blocks(const SwapBlocksParams& p, int num_pairs, int num_caches,
+                               cudaStream_t stream);
+
 cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_copy_blocks(const CopyBlocksParams& p, int num_pairs, int num_layers,
                                cudaStream_t stream);

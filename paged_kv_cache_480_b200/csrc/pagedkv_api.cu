@@ -405,6 +405,52 @@ pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_lay
     return PKV_OK;
 }
 
+pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, int num_caches,
+                       const int64_t* block_mapping, int num_pairs, int src_num_blocks,
+                       int dst_num_blocks, int64_t block_bytes, void* stream) {
+    if (num_caches < 0 || num_caches > 2 * pkv::kMaxLayers || num_pairs < 0 || src_num_blocks <= 0 ||
+        dst_num_blocks <= 0 || block_bytes <= 0 || block_bytes % 16 != 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_pairs == 0 || num_caches == 0) return PKV_OK;
+    if (!src_caches || !dst_caches || !block_mapping || (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    if (num_pairs > 65535) return PKV_ERR_UNSUPPORTED;
+    // Every buffer must be reachable from the device: device memory, or host
+    // memory that is pinned (page-locked) and mapped.
+    auto reachable = [](const void* ptr) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return true;
+        return a.type == cudaMemoryTypeHost && a.devicePointer == ptr;
+    };
+    pkv::SwapBlocksParams p;
+    std::memset(&p, 0, sizeof p);
+    for (int c = 0; c < num_caches; ++c) {
+        if (!src_caches[c] || !dst_caches[c] || !aligned16(src_caches[c]) || !aligned16(dst_caches[c]))
+            return PKV_ERR_INVALID_ARG;
+        if (!reachable(src_caches[c]) || !reachable(dst_caches[c])) return PKV_ERR_INVALID_ARG;
+        p.src[c] = src_caches[c];
+        p.dst[c] = dst_caches[c];
+    }
+    if (!reachable(block_mapping)) return PKV_ERR_INVALID_ARG;
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    pkv_status st = device_info(&sms, &errors);
+    if (st != PKV_OK) return st;
+    p.block_mapping = block_mapping;
+    p.errors = errors;
+    p.block_bytes = block_bytes;
+    p.src_blocks = src_num_blocks;
+    p.dst_blocks = dst_num_blocks;
+    if (pkv::launch_swap_blocks(p, num_pairs, num_caches, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
 pkv_status pkv_read_device_errors(void* stream, uint32_t* bits) {
     if (!bits) return PKV_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;

@@ -102,3 +102,35 @@ def test_errors():
     assert bm.num_free() == 3
     with pytest.raises(binding.PagedKVError):
         binding.BlockManager(4, 16, free_order=[0, 1, 1, 2])   # not a permutation
+
+
+def test_swap_out_and_in_match_model_exactly():
+    rng = np.random.default_rng(9)
+    g_order, h_order = rng.permutation(50), rng.permutation(18)
+    gpu, host = binding.BlockManager(50, 16, g_order), binding.BlockManager(18, 16, h_order)
+    mg, mh = BlockManagerModel(50, 16, g_order), BlockManagerModel(18, 16, h_order)
+    for bm, model in ((gpu, mg),):
+        for s, n in ((0, 70), (1, 33), (2, 100)):
+            bm.allocate(s, n)
+            model.allocate(s, n)
+        bm.fork(0, 3)
+        model.fork(0, 3)
+        assert bm.append_slot(3) == model.append_slot(3)
+    # swap out sequence 3 (shares 4 blocks with 0): private host copies
+    pairs = gpu.swap_out(host, 3)
+    want = mg.swap_out(3, mh)
+    assert [tuple(p) for p in pairs] == want
+    compare(gpu, mg, [0, 1, 2])
+    compare(host, mh, [3])
+    # all or nothing: sequences 2 (7 blocks) and 0 (5) fit in the 13 host blocks
+    # left; sequence 1 (3 blocks) then finds 1 free and must fail, changing nothing
+    for s in (2, 0):
+        assert [tuple(p) for p in gpu.swap_out(host, s)] == mg.swap_out(s, mh)
+    with pytest.raises(binding.OutOfBlocks):
+        gpu.swap_out(host, 1)
+    compare(gpu, mg, [1])
+    compare(host, mh, [0, 2, 3])
+    # swap back in
+    assert [tuple(p) for p in host.swap_out(gpu, 3)] == mh.swap_out(3, mg)
+    compare(gpu, mg, [1, 3])
+    compare(host, mh, [0, 2])

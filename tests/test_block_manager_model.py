@@ -150,3 +150,42 @@ def test_utilisation_bound_without_sharing():
     used = 400 - bm.num_free()
     assert bm.utilisation() == pytest.approx(lens.sum() / (used * 16))
     assert bm.utilisation() >= 1 - 15 * 20 / (used * 16)
+
+
+def test_swap_out_and_in_keep_contents_and_are_all_or_nothing():
+    rng = np.random.default_rng(7)
+    gpu = BlockManagerModel(40, 16, free_order=rng.permutation(40))
+    cpu = BlockManagerModel(10, 16)
+    sim = ContentSim(gpu)
+    sim.allocate(0, 70)
+    sim.fork(0, 1)
+    sim.append(1)                 # 71 tokens, last block copied on write
+    sim.allocate(2, 100)          # 7 blocks
+    pairs = gpu.swap_out(1, cpu)
+    assert len(pairs) == 5 and 1 not in gpu.tables and cpu.lens[1] == 71
+    host = {}
+    for gb, cb in pairs:          # the copies the caller makes
+        for off in range(16):
+            if gb * 16 + off in sim.slots:
+                host[cb * 16 + off] = sim.slots[gb * 16 + off]
+    hist1 = sim.history.pop(1)
+    gpu.check_invariants()
+    cpu.check_invariants()
+    sim.check()                   # the sequences left on the GPU are untouched
+    # all or nothing: sequence 2 needs 7 host blocks, 5 are free
+    before = copy.deepcopy((gpu.__dict__, cpu.__dict__))
+    with pytest.raises(OutOfBlocks):
+        gpu.swap_out(2, cpu)
+    assert (gpu.__dict__, cpu.__dict__) == before
+    # swap back in: fresh device blocks receive the host copies
+    back = gpu.swap_in(1, cpu)
+    assert len(back) == 5
+    for cb, gb in back:
+        for off in range(16):
+            if cb * 16 + off in host:
+                sim.slots[gb * 16 + off] = host[cb * 16 + off]
+    sim.history[1] = hist1
+    sim.check()                   # sequence 1 reads back exactly its history
+    assert cpu.num_free() == 10 and 1 not in cpu.tables
+    gpu.check_invariants()
+    cpu.check_invariants()

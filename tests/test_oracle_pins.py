@@ -366,3 +366,16 @@ def test_page_figures():
     p = g["pages_for_2048_tokens_at_128"]
     assert -(-p["tokens"] // p["page_size"]) == p["pages"]
     assert wl.CONFIGS["opt13b_f16"]["block_size"] == g["tokens_per_page_default"]["tokens"]
+
+
+def test_swap_blocks_matches_fancy_indexing():
+    rng = np.random.default_rng(18)
+    src = [rng.integers(0, 65535, (9, 2, 16, 8)).astype(np.uint16) for _ in range(2)]
+    dst = [rng.integers(0, 65535, (5, 2, 16, 8)).astype(np.uint16) for _ in range(2)]
+    mapping = np.array([[8, 0], [3, 4], [0, 2]], np.int64)
+    ref = [d.copy() for d in dst]
+    for s_, r in zip(src, ref):
+        r[mapping[:, 1]] = s_[mapping[:, 0]]
+    oracle.swap_blocks(src, dst, mapping)
+    for d, r in zip(dst, ref):
+        assert np.array_equal(d, r)
