@@ -46,6 +46,15 @@ def _load():
         lib.orc_copy_blocks.argtypes = [P, I, P, I, I64]
         lib.orc_swap_blocks.argtypes = [P, P, I, P, I, I64]
         lib.orc_round.argtypes = [P, P, I, I64]
+        lib.orc_paged_attention_ex.argtypes = [P, P, I, P, P, I, D, D, P, I, P, I, I, I, I, I, D, I]
+        lib.orc_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.orc_e4m3_to_double.restype = D
+        lib.orc_double_to_e4m3.argtypes = [D]
+        lib.orc_double_to_e4m3.restype = ctypes.c_uint8
+        lib.orc_quantize_e4m3.argtypes = [D, ctypes.c_float]
+        lib.orc_quantize_e4m3.restype = ctypes.c_uint8
+        lib.orc_reshape_and_cache_e4m3.argtypes = [P, P, I, P, P, P, I, I, I, I, I64, I64,
+                                                   ctypes.c_float, ctypes.c_float]
         lib.orc_load.argtypes = [P, I, I64]
         lib.orc_load.restype = D
         lib.orc_double_to_f16.argtypes = [D]
@@ -205,3 +214,48 @@ def swap_blocks(src_pools, dst_pools, block_mapping):
     sa = (ctypes.c_void_p * n)(*[a.ctypes.data for a in src_pools])
     da = (ctypes.c_void_p * n)(*[a.ctypes.data for a in dst_pools])
     _load().orc_swap_blocks(sa, da, n, _ptr(bm), bm.shape[0], block_bytes)
+
+
+def e4m3_to_double(code):
+    return _load().orc_e4m3_to_double(int(code))
+
+
+def e4m3_bits(x):
+    return _load().orc_double_to_e4m3(float(x))
+
+
+def quantize_e4m3(x, scale):
+    """The cache code of x: e4m3(fp32(x) / fp32(scale))."""
+    return _load().orc_quantize_e4m3(float(x), ctypes.c_float(scale))
+
+
+def paged_attention_fp8(q, qdtype, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                        scale, num_kv_heads, block_size, nthreads=None):
+    """fp64 decode attention over E4M3 caches (uint8 codes) times their scales."""
+    qc = DTYPE_CODES[qdtype]
+    q = _raw(q, qc)
+    kc = np.ascontiguousarray(k_cache, dtype=np.uint8)
+    vc = np.ascontiguousarray(v_cache, dtype=np.uint8)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S, H, D = q.shape
+    out = np.zeros((S, H, D), np.float64)
+    _load().orc_paged_attention_ex(_ptr(out), _ptr(q), qc, _ptr(kc), _ptr(vc), 3, float(k_scale),
+                                   float(v_scale), _ptr(bt), bt.shape[1], _ptr(cl), S, H,
+                                   num_kv_heads, D, block_size, float(scale),
+                                   nthreads or default_threads())
+    return out
+
+
+def reshape_and_cache_fp8(k, v, src_dtype, k_cache, v_cache, slot_mapping, block_size, k_scale,
+                          v_scale):
+    """Host quantising scatter into uint8 E4M3 caches, in place."""
+    sc = DTYPE_CODES[src_dtype]
+    k = _raw(k, sc)
+    v = _raw(v, sc)
+    assert k_cache.dtype == np.uint8 and k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    T, Hkv, D = k.shape
+    _load().orc_reshape_and_cache_e4m3(_ptr(k), _ptr(v), sc, _ptr(k_cache), _ptr(v_cache), _ptr(sm),
+                                       T, Hkv, D, block_size, Hkv * D, Hkv * D,
+                                       ctypes.c_float(k_scale), ctypes.c_float(v_scale))

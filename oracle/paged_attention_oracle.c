@@ -45,6 +45,7 @@
 #define ORC_F32 0
 #define ORC_F16 1
 #define ORC_BF16 2
+#define ORC_E4M3 3   /* cache elements only: FP8 E4M3 times a per-tensor scale */
 
 /* ---------------------------------------------------------------------
  * Element decoding: exact widening of the stored formats to fp64.
@@ -70,6 +71,43 @@ static double orc_bf16_to_double(uint16_t bits) {
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* FP8 E4M3 (the OCP 8-bit floating-point format): 1 sign bit, 4 exponent
+ * bits with bias 7, 3 fraction bits; exponent field 0 holds subnormals
+ * (fraction * 2^-9); there is no infinity and S.1111.111 is NaN; the largest
+ * finite magnitude is 1.75 * 2^8 = 448. */
+double orc_e4m3_to_double(uint8_t bits) {
+    int sign = bits >> 7;
+    int expo = (bits >> 3) & 0xf;
+    int frac = bits & 0x7;
+    double v;
+    if (expo == 0xf && frac == 0x7)
+        return NAN;
+    if (expo == 0)
+        v = ldexp((double)frac, -9);
+    else
+        v = ldexp((double)(frac | 0x8), expo - 10);  /* 1.frac * 2^(expo-7) */
+    return sign ? -v : v;
+}
+
+/* Round to E4M3, nearest with ties to even, saturating: a magnitude that
+ * would round above 448 becomes 448; NaN stays NaN (0x7f). */
+uint8_t orc_double_to_e4m3(double x) {
+    if (isnan(x)) return 0x7f;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7e;
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);
+    int E = e2 - 1;
+    if (E < -6) E = -6;                              /* subnormal range */
+    double quantum = ldexp(1.0, E - 3);
+    double r = nearbyint(a / quantum);
+    long bits = ((long)(E + 7) << 3) + (long)r - 8;  /* carries into the next binade */
+    if (bits > 0x7e) bits = 0x7e;                    /* 448 < a rounds up past 448 */
+    return sign | (uint8_t)bits;
 }
 
 double orc_load(const void* base, int dtype, int64_t index) {
@@ -140,14 +178,21 @@ static int64_t orc_cache_index(const int32_t* table_row, int t, int kv_head, int
 
 /* Gather the K and V rows of tokens [t0, t1) of one sequence and KV head
  * into contiguous fp64 arrays [t1 - t0][head_size]. */
-static void orc_gather(double* K, double* V, const void* k_cache, const void* v_cache, int dtype,
-                       const int32_t* table_row, int t0, int t1, int kv_head,
-                       int num_kv_heads, int block_size, int head_size) {
+/* A cache element's real value: the stored element, or for E4M3 the stored
+ * code times the tensor's scale (exact in fp64). */
+static double orc_cache_value(const void* cache, int cdtype, int64_t idx, double cscale) {
+    if (cdtype == ORC_E4M3) return orc_e4m3_to_double(((const uint8_t*)cache)[idx]) * cscale;
+    return orc_load(cache, cdtype, idx);
+}
+
+static void orc_gather(double* K, double* V, const void* k_cache, const void* v_cache, int cdtype,
+                       double k_scale, double v_scale, const int32_t* table_row, int t0, int t1,
+                       int kv_head, int num_kv_heads, int block_size, int head_size) {
     for (int t = t0; t < t1; ++t)
         for (int d = 0; d < head_size; ++d) {
             int64_t idx = orc_cache_index(table_row, t, kv_head, d, num_kv_heads, block_size, head_size);
-            K[(int64_t)(t - t0) * head_size + d] = orc_load(k_cache, dtype, idx);
-            V[(int64_t)(t - t0) * head_size + d] = orc_load(v_cache, dtype, idx);
+            K[(int64_t)(t - t0) * head_size + d] = orc_cache_value(k_cache, cdtype, idx, k_scale);
+            V[(int64_t)(t - t0) * head_size + d] = orc_cache_value(v_cache, cdtype, idx, v_scale);
         }
 }
 
@@ -161,9 +206,10 @@ static void orc_gather(double* K, double* V, const void* k_cache, const void* v_
  * For an empty range m = -inf, l = 0, acc = 0.
  * ------------------------------------------------------------------- */
 static void orc_row(double* acc, double* m_out, double* l_out, double* weights,
-                    const void* q, const void* k_cache, const void* v_cache, int dtype,
-                    const int32_t* table_row, int t0, int t1, int s, int h,
-                    int num_heads, int num_kv_heads, int head_size, int block_size, double scale) {
+                    const void* q, int qdtype, const void* k_cache, const void* v_cache, int cdtype,
+                    double k_scale, double v_scale, const int32_t* table_row, int t0, int t1,
+                    int s, int h, int num_heads, int num_kv_heads, int head_size, int block_size,
+                    double scale) {
     int G = num_heads / num_kv_heads;
     int kv_head = h / G;
     int n = t1 - t0;
@@ -176,10 +222,10 @@ static void orc_row(double* acc, double* m_out, double* l_out, double* weights,
     double* V = (double*)malloc(sizeof(double) * (size_t)n * head_size);
     double* z = (double*)malloc(sizeof(double) * (size_t)n);
     double* qd = (double*)malloc(sizeof(double) * (size_t)head_size);
-    orc_gather(K, V, k_cache, v_cache, dtype, table_row, t0, t1, kv_head,
+    orc_gather(K, V, k_cache, v_cache, cdtype, k_scale, v_scale, table_row, t0, t1, kv_head,
                num_kv_heads, block_size, head_size);
     for (int d = 0; d < head_size; ++d)
-        qd[d] = orc_load(q, dtype, ((int64_t)s * num_heads + h) * head_size + d);
+        qd[d] = orc_load(q, qdtype, ((int64_t)s * num_heads + h) * head_size + d);
 
     double m = -INFINITY;
     for (int t = 0; t < n; ++t) {
@@ -211,22 +257,33 @@ static void orc_row(double* acc, double* m_out, double* l_out, double* weights,
  * q: [S, H, D]; caches: [NB, Hkv, bs, D]; out: fp64 [S, H, D].
  * Rows are independent, so they are spread over nthreads OpenMP threads.
  * ------------------------------------------------------------------- */
-void orc_paged_attention(double* out, const void* q, const void* k_cache, const void* v_cache,
-                         int dtype, const int32_t* block_tables, int max_blocks_per_seq,
-                         const int32_t* context_lens, int num_seqs, int num_heads,
-                         int num_kv_heads, int head_size, int block_size, double scale,
-                         int nthreads) {
+void orc_paged_attention_ex(double* out, const void* q, int qdtype, const void* k_cache,
+                            const void* v_cache, int cdtype, double k_scale, double v_scale,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_size, int block_size, double scale,
+                            int nthreads) {
     int64_t rows = (int64_t)num_seqs * num_heads;
 #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
     for (int64_t r = 0; r < rows; ++r) {
         int s = (int)(r / num_heads), h = (int)(r % num_heads);
         double m, l;
         double* o = out + r * head_size;
-        orc_row(o, &m, &l, NULL, q, k_cache, v_cache, dtype,
+        orc_row(o, &m, &l, NULL, q, qdtype, k_cache, v_cache, cdtype, k_scale, v_scale,
                 block_tables + (int64_t)s * max_blocks_per_seq, 0, context_lens[s], s, h,
                 num_heads, num_kv_heads, head_size, block_size, scale);
         for (int d = 0; d < head_size; ++d) o[d] = (l > 0.0) ? o[d] / l : 0.0;
     }
+}
+
+void orc_paged_attention(double* out, const void* q, const void* k_cache, const void* v_cache,
+                         int dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_size, int block_size, double scale,
+                         int nthreads) {
+    orc_paged_attention_ex(out, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0, block_tables,
+                           max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads,
+                           head_size, block_size, scale, nthreads);
 }
 
 /* Attention weights of one (s, h) row: weights[t] for t < context_lens[s]. */
@@ -237,7 +294,7 @@ void orc_attention_weights(double* weights, const void* q, const void* k_cache,
                            double scale) {
     double m, l;
     double* acc = (double*)malloc(sizeof(double) * (size_t)head_size);
-    orc_row(acc, &m, &l, weights, q, k_cache, v_cache, dtype,
+    orc_row(acc, &m, &l, weights, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0,
             block_tables + (int64_t)s * max_blocks_per_seq, 0, context_lens[s], s, h, num_heads,
             num_kv_heads, head_size, block_size, scale);
     free(acc);
@@ -263,7 +320,7 @@ void orc_partition_stats(double* acc, double* m, double* l, const void* q, const
         int L = context_lens[s];
         int t0 = p * partition_size;
         int t1 = t0 + partition_size < L ? t0 + partition_size : L;
-        orc_row(acc + r * head_size, m + r, l + r, NULL, q, k_cache, v_cache, dtype,
+        orc_row(acc + r * head_size, m + r, l + r, NULL, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0,
                 block_tables + (int64_t)s * max_blocks_per_seq, t0, t1, s, h, num_heads,
                 num_kv_heads, head_size, block_size, scale);
     }
@@ -351,4 +408,36 @@ void orc_swap_blocks(void** src_pools, void** dst_pools, int num_caches, const i
         for (int i = 0; i < num_pairs; ++i)
             memcpy((char*)dst_pools[c] + mapping[2 * i + 1] * block_bytes,
                    (const char*)src_pools[c] + mapping[2 * i] * block_bytes, (size_t)block_bytes);
+}
+
+/* ---------------------------------------------------------------------------
+ * Cache write into an E4M3 cache: code = e4m3(fp32(x) / fp32(scale)), the
+ * quotient correctly rounded in fp32 (the precision the kernel takes the
+ * decision in), then rounded to E4M3 as orc_double_to_e4m3 does.
+ * k, v: [T][...] in src_dtype with key_stride / value_stride elements between
+ * tokens; caches: uint8 [NB][Hkv][bs][D].
+ * ------------------------------------------------------------------- */
+uint8_t orc_quantize_e4m3(double x, float scale) {
+    float q = (float)x / scale;          /* x is exact in fp32 for every source format */
+    return orc_double_to_e4m3((double)q);
+}
+
+void orc_reshape_and_cache_e4m3(const void* k, const void* v, int src_dtype, uint8_t* k_cache,
+                                uint8_t* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                int num_kv_heads, int head_size, int block_size,
+                                int64_t key_stride, int64_t value_stride, float k_scale,
+                                float v_scale) {
+    for (int i = 0; i < num_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0) continue;
+        int64_t b = slot / block_size, off = slot % block_size;
+        for (int g = 0; g < num_kv_heads; ++g)
+            for (int d = 0; d < head_size; ++d) {
+                int64_t dst = ((b * num_kv_heads + g) * block_size + off) * head_size + d;
+                k_cache[dst] = orc_quantize_e4m3(
+                    orc_load(k, src_dtype, (int64_t)i * key_stride + (int64_t)g * head_size + d), k_scale);
+                v_cache[dst] = orc_quantize_e4m3(
+                    orc_load(v, src_dtype, (int64_t)i * value_stride + (int64_t)g * head_size + d), v_scale);
+            }
+    }
 }
