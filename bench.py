@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--measure", default="decode", choices=["decode", "swap"],
                     help="swap: swap_blocks between the GPU pool and a pinned host pool")
+    ap.add_argument("--kv-cache", default="auto", choices=["auto", "fp8"],
+                    help="fp8: E4M3 cache written by reshape_and_cache_fp8kv, read by the fp8 decode")
     ap.add_argument("--fused", action="store_true",
                     help="cache write fused into the decode (paged_attention_decode_append)")
     return ap.parse_args()
@@ -61,31 +63,43 @@ def peaks():
 # ---------------------------------------------------------------------------
 # workload and byte model
 # ---------------------------------------------------------------------------
-def decode_bytes(lay):
+def decode_bytes(lay, cache_bytes=None):
     """Algorithmic bytes of one decode call: K+V of every context token, q
-    and out, the block-table entries read and the context lengths."""
+    and out, the block-table entries read and the context lengths.
+    cache_bytes: bytes per cache element (default: the model's dtype)."""
     from paged_kv_cache_480_b200.workloads import DTYPE_BYTES
     dt = DTYPE_BYTES[lay.dtype]
+    cb = dt if cache_bytes is None else cache_bytes
     lens = lay.context_lens.astype(np.int64)
-    kv = int(lens.sum()) * lay.num_kv_heads * lay.head_size * dt * 2
+    kv = int(lens.sum()) * lay.num_kv_heads * lay.head_size * cb * 2
     qo = 2 * lay.num_seqs * lay.num_heads * lay.head_size * dt
     tables = int((-(-lens // lay.block_size)).sum()) * 4
     return kv + qo + tables + 4 * lay.num_seqs
 
 
-def cache_write_bytes(lay):
+def cache_write_bytes(lay, cache_bytes=None):
     """reshape_and_cache of one token per sequence: read k, v; write them; read slots."""
     from paged_kv_cache_480_b200.workloads import DTYPE_BYTES
-    row = lay.num_kv_heads * lay.head_size * DTYPE_BYTES[lay.dtype]
-    return lay.num_seqs * (4 * row + 8)
+    dt = DTYPE_BYTES[lay.dtype]
+    cb = dt if cache_bytes is None else cache_bytes
+    n = lay.num_kv_heads * lay.head_size
+    return lay.num_seqs * (2 * n * dt + 2 * n * cb + 8)
 
 
-def build_workload(name, block_size, device):
+FP8_SCALES = (1.0 / 64, 1.0 / 64)
+
+
+def build_workload(name, block_size, device, fp8=False):
     from paged_kv_cache_480_b200 import workloads as wl
     if name == "cow_bf16":
+        if fp8:
+            raise SystemExit("--kv-cache fp8 runs the decode workloads only")
         return build_cow_state(device)
     lay = wl.make_layout(name, block_size=block_size)
-    ten = wl.make_tensors(lay, device=device)
+    if fp8:
+        ten = wl.make_tensors_fp8(lay, device=device, k_scale=FP8_SCALES[0], v_scale=FP8_SCALES[1])
+    else:
+        ten = wl.make_tensors(lay, device=device)
     return lay, ten, None
 
 
@@ -327,7 +341,11 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     pkv.load_library()
-    lay, ten, pairs = build_workload(args.workload, args.block_size, device)
+    fp8 = args.kv_cache == "fp8"
+    if fp8 and args.fused:
+        raise SystemExit("--fused works with caches of the model's dtype")
+    cb = 1 if fp8 else None
+    lay, ten, pairs = build_workload(args.workload, args.block_size, device, fp8)
     S, H, Hkv, D, bs = lay.num_seqs, lay.num_heads, lay.num_kv_heads, lay.head_size, lay.block_size
     max_ctx = lay.max_context_len
     bt = torch.from_numpy(lay.block_tables).to(device)
@@ -349,14 +367,21 @@ def run_ours(args, rank, world, local_rank):
     def step(record=False):
         if pairs_d is not None:
             pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], pairs_d, stream=stream)
-        if not args.fused:
+        if fp8:
+            pkv.reshape_and_cache_fp8kv(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm,
+                                        *FP8_SCALES, stream=stream)
+        elif not args.fused:
             pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm,
                                   stream=stream)
         if record:
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-        if args.fused:
+        if fp8:
+            pkv.paged_attention_decode_fp8kv(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl,
+                                             lay.scale, *FP8_SCALES, max_context_len=max_ctx,
+                                             partition_size=ps, workspace=ws, stream=stream)
+        elif args.fused:
             pkv.paged_attention_decode_append(out, ten["q"], ten["k_new"], ten["v_new"], ten["k_cache"],
                                               ten["v_cache"], sm, bt, cl, lay.scale,
                                               max_context_len=max_ctx, partition_size=ps,
@@ -393,7 +418,7 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = [a.elapsed_time(b) for a, b in ev]
     errors = pkv.read_device_errors()
 
-    step_bytes = decode_bytes(lay) + cache_write_bytes(lay)
+    step_bytes = decode_bytes(lay, cb) + cache_write_bytes(lay, cb)
     if pairs_d is not None:
         step_bytes += 2 * len(pairs) * 2 * Hkv * bs * D * 2
     ms_step = ms_total / args.steps
@@ -403,21 +428,22 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         peak, peak_kind = peaks()
         dec_avg = sum(dec_ms) / len(dec_ms)
-        achieved = decode_bytes(lay) / (dec_avg * 1e-3) / 1e9
+        achieved = decode_bytes(lay, cb) / (dec_avg * 1e-3) / 1e9
         kname = "paged_attention_decode_append (fused cache write + decode" if args.fused else \
-            "paged_attention_decode (decode"
+            "paged_attention_decode_fp8kv (decode" if fp8 else "paged_attention_decode (decode"
         roof = {"kernel": kname + (" + lse merge)" if split else ")"),
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind,
                 "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
-                "traffic": profiled_traffic(lay.name, bs), "algorithmic_bytes": decode_bytes(lay),
+                "traffic": None if fp8 else profiled_traffic(lay.name, bs),
+                "algorithmic_bytes": decode_bytes(lay, cb),
                 "avg_call_us": dec_avg * 1e3}
         result = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
                   "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                   "us_per_step": ms_step * 1e3, "seqs_per_s": world * S / (ms_step * 1e-3),
                   "pct_of_peak": 100 * value / world / peak,
                   "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                  "dtype": lay.dtype, "data": "synthetic",
+                  "dtype": lay.dtype + ("/fp8-e4m3 cache" if fp8 else ""), "data": "synthetic",
                   "config": {"workload": lay.name, "num_seqs": S, "num_heads": H,
                              "num_kv_heads": Hkv, "head_size": D, "block_size": bs,
                              "num_blocks": lay.num_blocks, "max_context_len": max_ctx,
@@ -425,13 +451,14 @@ def run_ours(args, rank, world, local_rank):
                              "partition_size": nparts, "split_context": split,
                              "cow_pairs": 0 if pairs is None else int(len(pairs)),
                              "step_bytes": step_bytes, "fused_cache_write": bool(args.fused),
+                             "kv_cache": "fp8-e4m3" if fp8 else lay.dtype,
                              "l2": f"inputs larger than L2: {lay.kv_bytes() / 1e9:.2f} GB of K/V per step",
                              "parallelism": f"replicas x{world}"},
                   "roofline": roof, "gpu_launches": launches_per_step * args.steps,
                   "clocks": clk.summary(), "device_errors": errors}
-        if not args.no_e2e:
+        if not args.no_e2e and not fp8:
             result["e2e"] = run_e2e(args, lay, ten, pairs, device, ws, step_bytes)
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and not fp8:
             host = host_arrays(ten, lay.dtype)
             gbs, t, b, seqs, threads = oracle_sample(lay, host, 10.0,
                                                      max_seqs=max(1, lay.num_seqs // 8))

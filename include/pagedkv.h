@@ -155,6 +155,44 @@ pkv_status paged_attention_decode_append(void* out, const void* q, const void* k
                                          pkv_dtype dtype, int partition_size, void* workspace,
                                          size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * FP8 KV cache ("GPT-OSS memory management: PagedAttention explained",
+ * section 3.2: kv_cache_dtype configures the cache element type).
+ *
+ * The caches hold FP8 E4M3 codes (1 byte per element: 1 sign, 4 exponent bits
+ * with bias 7, 3 fraction bits, no infinities, 0x7f/0xff NaN, largest finite
+ * 448), same layout [num_blocks][num_kv_heads][block_size][head_size], and a
+ * cache element stands for code * scale with one scale for all of K
+ * (k_scale) and one for all of V (v_scale), both > 0.
+ *
+ * paged_attention_decode_fp8kv: paged_attention_decode over such caches:
+ *   out[s, h, :] = sum_t softmax_t(scale * q . (k_scale * K_s[t])) v_scale * V_s[t],
+ * q and out in `dtype` (f32, f16 or bf16).  Workspace, partitioning, checks
+ * and errors as for paged_attention_decode (the workspace size does not
+ * depend on the cache type).  With 16-bit q and 4 or 8 query heads per KV
+ * head the products run on the tensor cores in fp16 (E4M3 is exact in fp16;
+ * bf16 q is rounded to fp16 there, so |q| must stay below 65504).
+ *
+ * reshape_and_cache_fp8kv: reshape_and_cache into such caches: each element
+ * x of key (value) becomes e4m3(x / k_scale) (resp. v_scale), the quotient
+ * correctly rounded in fp32 and then rounded to nearest-even E4M3,
+ * saturating to +-448 (NaN stays NaN).  key/value are in `dtype`.
+ * ------------------------------------------------------------------------- */
+pkv_status paged_attention_decode_fp8kv(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const int32_t* block_tables,
+                                        const int32_t* context_lens, float scale, float k_scale,
+                                        float v_scale, int num_kv_heads, int block_size,
+                                        int num_seqs, int num_heads, int head_size, int num_blocks,
+                                        int max_blocks_per_seq, int max_context_len,
+                                        pkv_dtype dtype, int partition_size, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+pkv_status reshape_and_cache_fp8kv(const void* key, const void* value, void* k_cache,
+                                  void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                  int num_kv_heads, int head_size, int block_size, int num_blocks,
+                                  int64_t key_token_stride, int64_t value_token_stride,
+                                  pkv_dtype dtype, float k_scale, float v_scale, void* stream);
+
 /* Bytes of workspace paged_attention_decode needs for these sizes (0 on bad
  * arguments).  partition_size as in paged_attention_decode. */
 size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

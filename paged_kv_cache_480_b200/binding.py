@@ -69,6 +69,11 @@ def load_library(path=LIB_PATH):
         lib.swap_blocks.restype = I
         lib.pkv_bm_swap_out.argtypes = [P, P, I64, P, I, ctypes.POINTER(I)]
         lib.pkv_bm_swap_out.restype = I
+        lib.paged_attention_decode_fp8kv.argtypes = [P, P, P, P, P, P, F, F, F, I, I, I, I, I, I, I, I,
+                                                     I, I, P, SZ, P]
+        lib.paged_attention_decode_fp8kv.restype = I
+        lib.reshape_and_cache_fp8kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I64, I64, I, F, F, P]
+        lib.reshape_and_cache_fp8kv.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         lib.pkv_read_device_errors.restype = I
         lib.pkv_bm_create.argtypes = [I, I, P, ctypes.POINTER(P)]
@@ -248,6 +253,65 @@ def paged_attention_decode_append(out, q, key, value, k_cache, v_cache, slot_map
         workspace.numel() * workspace.element_size(), _stream(stream, q.device))
     _check(st, "paged_attention_decode_append")
     return out
+
+
+def _fp8_cache(t, name):
+    import torch
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    return _contig(t, name)
+
+
+def paged_attention_decode_fp8kv(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                 k_scale, v_scale, max_context_len=None, partition_size=0,
+                                 workspace=None, stream=None):
+    """Decode attention over FP8 E4M3 caches (paged_attention_decode_fp8kv in
+    pagedkv.h): k_cache / v_cache uint8 [NB, Hkv, bs, D]; q, out in f32/f16/bf16."""
+    import torch
+    lib = load_library()
+    S, H, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("shape / dtype mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    MB = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = MB * bs
+    code = _dtype_code(q)
+    need = lib.paged_attention_workspace_size(S, H, Hkv, D, bs, max_context_len, code, partition_size)
+    if need == 0:
+        raise PagedKVError(2, "paged_attention_workspace_size")
+    if workspace is None:
+        workspace = default_workspace(q.device, need)
+    st = lib.paged_attention_decode_fp8kv(
+        _contig(out, "out"), _contig(q, "q"), _fp8_cache(k_cache, "k_cache"), _fp8_cache(v_cache, "v_cache"),
+        _contig(block_tables, "block_tables"), _contig(context_lens, "context_lens"), float(scale),
+        float(k_scale), float(v_scale), Hkv, bs, S, H, D, NB, MB, int(max_context_len), code,
+        int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream, q.device))
+    _check(st, "paged_attention_decode_fp8kv")
+    return out
+
+
+def reshape_and_cache_fp8kv(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None):
+    """Quantising cache write into FP8 E4M3 caches (reshape_and_cache_fp8kv in pagedkv.h)."""
+    import torch
+    lib = load_library()
+    T, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv, D) != (Hkv2, D2) or value.shape != key.shape:
+        raise ValueError("key/value shape does not match the cache")
+    if key.stride(2) != 1 or key.stride(1) != D or value.stride(2) != 1 or value.stride(1) != D:
+        raise ValueError("key/value heads must be contiguous within a token")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T:
+        raise TypeError("slot_mapping must be int64 [T]")
+    st = lib.reshape_and_cache_fp8kv(
+        _cuda(key, "key"), _cuda(value, "value"), _fp8_cache(k_cache, "k_cache"),
+        _fp8_cache(v_cache, "v_cache"), _contig(slot_mapping, "slot_mapping"), T, Hkv, D, bs, NB,
+        key.stride(0), value.stride(0), _dtype_code(key), float(k_scale), float(v_scale),
+        _stream(stream, key.device))
+    _check(st, "reshape_and_cache_fp8kv")
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

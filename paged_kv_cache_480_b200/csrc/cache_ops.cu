@@ -109,6 +109,71 @@ cudaError_t launch_swap_blocks(const SwapBlocksParams& p, int num_pairs, int num
     return launch_pdl(swap_blocks_kernel, dim3(num_pairs, num_caches), dim3(256), 0, stream, p);
 }
 
+// Cache write into an FP8 (E4M3) cache: each element becomes
+// e4m3(x / scale) -- the quotient correctly rounded in fp32, then rounded to
+// nearest-even E4M3 with saturation at +-448.  One thread per 16 output
+// bytes (16 elements) of one (token, KV head) row.
+template <typename TS>
+__global__ void reshape_and_cache_fp8_kernel(const CacheWriteFp8Params p) {
+    griddep_wait();
+    griddep_launch();
+    constexpr int EPS = Elem<TS>::kPerChunk;      // source elements per 16 bytes
+    const int64_t chunks_per_row = p.head_size / 16;
+    const int64_t per_token = (int64_t)p.num_kv_heads * chunks_per_row;
+    const int64_t total = (int64_t)p.num_tokens * per_token;
+    const int64_t pool_slots = (int64_t)p.num_blocks * p.block_size;
+    for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
+         w += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = w / per_token;
+        const int64_t rem = w - i * per_token;
+        const int64_t g = rem / chunks_per_row;
+        const int64_t ch = rem - g * chunks_per_row;
+        const int64_t slot = p.slot_mapping[i];
+        if (slot < 0) continue;
+        if (slot >= pool_slots) {
+            if (rem == 0) flag_error(p.errors, PKV_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / p.block_size, off = slot - blk * p.block_size;
+        const int64_t dst = ((blk * p.num_kv_heads + g) * p.block_size + off) * p.head_size + ch * 16;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const TS* src = reinterpret_cast<const TS*>(which ? p.value : p.key) +
+                            i * (which ? p.value_stride : p.key_stride) + g * p.head_size + ch * 16;
+            const float sc = which ? p.v_scale : p.k_scale;
+            float x[16];
+#pragma unroll
+            for (int k = 0; k < 16 / EPS; ++k)
+                Elem<TS>::widen(reinterpret_cast<const uint4*>(src)[k], x + k * EPS);
+            uint32_t out[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(x[4 * k], sc), __fdiv_rn(x[4 * k + 1], sc));
+                const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(x[4 * k + 2], sc), __fdiv_rn(x[4 * k + 3], sc));
+                out[k] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+            *reinterpret_cast<uint4*>((which ? p.v_cache : p.k_cache) + dst) =
+                make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    }
+}
+
+cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Params& p, int num_sms,
+                                         cudaStream_t stream) {
+    const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.head_size / 16);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    const int64_t cap = (int64_t)num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    const dim3 grid((unsigned)blocks), block(threads);
+    switch (p.src_dtype) {
+        case PKV_F32: return launch_pdl(reshape_and_cache_fp8_kernel<float>, grid, block, 0, stream, p);
+        case PKV_F16: return launch_pdl(reshape_and_cache_fp8_kernel<__half>, grid, block, 0, stream, p);
+        default: return launch_pdl(reshape_and_cache_fp8_kernel<__nv_bfloat16>, grid, block, 0, stream, p);
+    }
+}
+
 cudaError_t launch_reshape_and_cache(const CacheWriteParams& p, int num_sms, cudaStream_t stream) {
     const int64_t total = (int64_t)p.num_tokens * p.num_kv_heads * (p.row_bytes / 16);
     if (total == 0) return cudaSuccess;

@@ -39,6 +39,22 @@ struct SwapBlocksParams {
     int64_t src_blocks, dst_blocks;
 };
 
+struct CacheWriteFp8Params {
+    const void* key;
+    const void* value;
+    unsigned char* k_cache;        // E4M3 bytes, [NB][Hkv][bs][D]
+    unsigned char* v_cache;
+    const int64_t* slot_mapping;
+    unsigned int* errors;
+    int64_t key_stride, value_stride;   // elements between tokens
+    float k_scale, v_scale;
+    int num_tokens, num_kv_heads, head_size, block_size, num_blocks;
+    int src_dtype;                 // pkv_dtype of key / value
+};
+
+cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Params& p, int num_sms,
+                                         cudaStream_t stream);
+
 cudaError_t launch_swap_blocks(const SwapBlocksParams& p, int num_pairs, int num_caches,
                                cudaStream_t stream);
 

@@ -80,6 +80,48 @@ template <> struct Elem<__half> {
     }
 };
 
+// FP8 E4M3 cache elements (1 sign, 4 exponent bits with bias 7, 3 fraction
+// bits; no infinities, 0x7f/0xff are NaN, largest finite 448).  Stored
+// values are the real values divided by a per-tensor scale.
+struct fp8e4m3 {
+    uint8_t bits;
+};
+
+// Two E4M3 values (low byte -> low half) to two exact fp16 values.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+    return h;
+}
+
+// Round two fp32 values to E4M3 (nearest, ties to even; beyond +-448 they
+// saturate to +-448): lo -> low byte, hi -> high byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t v;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(v) : "f"(hi), "f"(lo));
+    return v;
+}
+
+template <> struct Elem<fp8e4m3> {
+    static constexpr int kPerChunk = 16;
+    __device__ __forceinline__ static void widen4(uint32_t w, float* f) {
+        const uint32_t ha = e4m3x2_to_f16x2((uint16_t)(w & 0xffffu));
+        const uint32_t hb = e4m3x2_to_f16x2((uint16_t)(w >> 16));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&ha));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hb));
+        f[0] = a.x;
+        f[1] = a.y;
+        f[2] = b.x;
+        f[3] = b.y;
+    }
+    __device__ __forceinline__ static void widen(const uint4& c, float* f) {
+        widen4(c.x, f);
+        widen4(c.y, f + 4);
+        widen4(c.z, f + 8);
+        widen4(c.w, f + 12);
+    }
+};
+
 // ---------------------------------------------------------------------------
 // Shared-memory and bulk-copy (TMA, untiled) primitives.
 // ---------------------------------------------------------------------------

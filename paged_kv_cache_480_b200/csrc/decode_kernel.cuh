@@ -48,6 +48,7 @@ struct DecodeParams {
     int32_t* prefix_out;    // [S + 1] partitions before each sequence
     unsigned int* errors;   // sticky device-check bits
     float scale_log2;       // scale * log2(e)
+    float k_scale, v_scale; // cache element = real value / scale (1 unless the cache is FP8)
     int num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq, max_context_len;
     int partition_size;     // PS tokens, a multiple of block_size, <= 32 blocks
     int partition_min;      // > 0: choose PS in [partition_min, partition_size] on the device
@@ -64,12 +65,14 @@ struct DecodeParams {
     uint32_t seq_smem;      // bytes of the per-CTA length / prefix arrays
 };
 
-template <typename T, int D, int BS, int G>
+// TQ: element type of q and out; TC: element type of the caches.
+template <typename TQ, typename TC, int D, int BS, int G>
 struct DecodeShape {
-    static constexpr int EPC = Elem<T>::kPerChunk;  // elements per 16-byte chunk
-    static constexpr int ROW = D * (int)sizeof(T);  // bytes per token row
-    static constexpr int TILE = BS * ROW;           // bytes per (block, KV head) tile
-    static constexpr int QBYTES = G * ROW;          // q rows of one group
+    static constexpr int EPC = Elem<TC>::kPerChunk;  // cache elements per 16-byte chunk
+    static constexpr int ROW = D * (int)sizeof(TC);  // bytes per cache token row
+    static constexpr int TILE = BS * ROW;            // bytes per (block, KV head) tile
+    static constexpr int QROW = D * (int)sizeof(TQ); // bytes per q / out row
+    static constexpr int QBYTES = G * QROW;          // q rows of one group
 };
 
 struct StageMeta {
@@ -84,9 +87,9 @@ struct StageMeta {
 constexpr int kFirst = 1, kLast = 2, kWhole = 4;
 
 // Host and device agree on this layout of one warp's shared-memory region.
-template <typename T, int D, int BS, int G>
+template <typename TQ, typename TC, int D, int BS, int G>
 struct WarpSmem {
-    using S = DecodeShape<T, D, BS, G>;
+    using S = DecodeShape<TQ, TC, D, BS, G>;
     __host__ __device__ static constexpr uint32_t ring(int) { return 0; }
     __host__ __device__ static constexpr uint32_t qbuf(int R) { return (uint32_t)R * 2 * S::TILE; }
     // new-token K and V rows of each stage (fused cache write)
@@ -131,12 +134,15 @@ constexpr unsigned kFull = 0xffffffffu;
 // lanes of a quarter-warp read one 128-byte segment of a row (no bank
 // conflicts).
 // ===========================================================================
-template <typename T, int D, int BS, int G>
+template <typename TQ, typename TC, int D, int BS, int G>
 struct FmaConsumer {
-    using S = DecodeShape<T, D, BS, G>;
+    using S = DecodeShape<TQ, TC, D, BS, G>;
     static constexpr int EPC = S::EPC;
+    static constexpr int EPQ = Elem<TQ>::kPerChunk;  // q / out elements per 16-byte chunk
+    static constexpr int QPC = EPC / EPQ;           // q chunks per cache chunk
     static constexpr int NCH = D / EPC;             // chunks per token row
-    static constexpr int Q = (G >= 8) ? 4 : 8;      // lanes per token row
+    static constexpr int Q0 = (G >= 8) ? 4 : 8;
+    static constexpr int Q = Q0 < NCH ? Q0 : NCH;   // lanes per token row
     static constexpr int CPL = NCH / Q;             // chunks per lane
     static constexpr int DL = CPL * EPC;            // dims per lane
     static constexpr int TS = 32 / (Q * G);         // token rows per warp step
@@ -158,15 +164,17 @@ struct FmaConsumer {
         for (int d = 0; d < DL; ++d) qf[d] = acc[d] = 0.f;
     }
 
-    __device__ __forceinline__ void begin(const unsigned char* qslot, float scale_log2) {
-        const uint4* qrow = reinterpret_cast<const uint4*>(qslot + h * S::ROW);
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float qscale) {
+        const uint4* qrow = reinterpret_cast<const uint4*>(qslot + h * S::QROW);
 #pragma unroll
-        for (int k = 0; k < CPL; ++k) {
-            float f[EPC];
-            Elem<T>::widen(qrow[c + Q * k], f);
+        for (int k = 0; k < CPL; ++k)
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) qf[k * EPC + e] = f[e] * scale_log2;
-        }
+            for (int j = 0; j < QPC; ++j) {
+                float f[EPQ];
+                Elem<TQ>::widen(qrow[(c + Q * k) * QPC + j], f);
+#pragma unroll
+                for (int e = 0; e < EPQ; ++e) qf[k * EPC + j * EPQ + e] = f[e] * qscale;
+            }
 #pragma unroll
         for (int d = 0; d < DL; ++d) acc[d] = 0.f;
         m_run = -INFINITY;
@@ -184,7 +192,7 @@ struct FmaConsumer {
 #pragma unroll
             for (int k = 0; k < CPL; ++k) {
                 float f[EPC];
-                Elem<T>::widen(row[c + Q * k], f);
+                Elem<TC>::widen(row[c + Q * k], f);
 #pragma unroll
                 for (int e = 0; e < EPC; e += 2) {
                     s0 = fmaf(qf[k * EPC + e], f[e], s0);
@@ -216,7 +224,7 @@ struct FmaConsumer {
 #pragma unroll
                 for (int k = 0; k < CPL; ++k) {
                     float f[EPC];
-                    Elem<T>::widen(row[c + Q * k], f);
+                    Elem<TC>::widen(row[c + Q * k], f);
 #pragma unroll
                     for (int e = 0; e < EPC; ++e) acc[k * EPC + e] = fmaf(pr, f[e], acc[k * EPC + e]);
                 }
@@ -235,25 +243,28 @@ struct FmaConsumer {
         }
         if (u != 0) return;
         if (mt.flags & kWhole) {
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) +
+            const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
+            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<TQ*>(p.out) +
                                                    ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + h) * D);
 #pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                float f[EPC];
+            for (int k = 0; k < CPL; ++k)
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) f[e] = acc[k * EPC + e] * inv;
-                orow[c + Q * k] = Elem<T>::narrow(f);
-            }
+                for (int j = 0; j < QPC; ++j) {
+                    float f[EPQ];
+#pragma unroll
+                    for (int e = 0; e < EPQ; ++e) f[e] = acc[k * EPC + j * EPQ + e] * inv;
+                    orow[(c + Q * k) * QPC + j] = Elem<TQ>::narrow(f);
+                }
         } else {
+            const float vs = p.v_scale;
             float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + h) * D);
 #pragma unroll
             for (int k = 0; k < CPL; ++k)
 #pragma unroll
                 for (int e = 0; e < EPC; e += 4)
                     prow[((c + Q * k) * EPC + e) / 4] =
-                        make_float4(acc[k * EPC + e], acc[k * EPC + e + 1], acc[k * EPC + e + 2],
-                                    acc[k * EPC + e + 3]);
+                        make_float4(acc[k * EPC + e] * vs, acc[k * EPC + e + 1] * vs,
+                                    acc[k * EPC + e + 2] * vs, acc[k * EPC + e + 3] * vs);
             if (c == 0) p.part_ml[(size_t)mt.item * G + h] = make_float2(m_run, lt);
         }
     }
@@ -278,9 +289,9 @@ struct FmaConsumer {
 // ===========================================================================
 template <typename T, int D, int BS, int G>
 struct MmaConsumer {
-    using S = DecodeShape<T, D, BS, G>;
+    using S = DecodeShape<T, T, D, BS, G>;
     static_assert(sizeof(T) == 2, "tensor-core consumer needs 16-bit elements");
-    static_assert(G == 4 || G == 8, "tensor-core consumer serves groups of 4 or 8 heads");
+    static_assert(G <= 8, "the 8 MMA columns hold the query heads of one group");
     static constexpr int KJ = D / 32;      // 16-byte chunks per lane per K row
     static constexpr int MT = D / 16;      // PV MMAs (row tiles of 16 dims)
     static constexpr int VCH = D / 64;     // 16-byte chunks per lane per V row (D/8 dims)
@@ -448,7 +459,7 @@ struct MmaConsumer {
             if (head >= G) continue;
             const float lt = e ? t1 : t0;
             if (mt.flags & kWhole) {
-                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
                 uint32_t words[MT];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) words[m] = Elem<T>::pack2(o[m][e] * inv, o[m][2 + e] * inv);
@@ -460,11 +471,13 @@ struct MmaConsumer {
                     orow[ch] = make_uint4(words[4 * ch], words[4 * ch + 1], words[4 * ch + 2],
                                           words[4 * ch + 3]);
             } else {
+                const float vs = p.v_scale;
                 float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + head) * D +
                                                          r * (D / 8));
 #pragma unroll
                 for (int m = 0; m < MT; m += 2)
-                    prow[m / 2] = make_float4(o[m][e], o[m][2 + e], o[m + 1][e], o[m + 1][2 + e]);
+                    prow[m / 2] = make_float4(o[m][e] * vs, o[m][2 + e] * vs, o[m + 1][e] * vs,
+                                              o[m + 1][2 + e] * vs);
                 if (r == 0)
                     p.part_ml[(size_t)mt.item * G + head] = make_float2(e ? m1 : m0, lt);
             }
@@ -472,14 +485,237 @@ struct MmaConsumer {
     }
 };
 
-template <typename T, int G>
-struct UseMma {
-    static constexpr bool value = sizeof(T) == 2 && (G == 4 || G == 8);
+// ===========================================================================
+// Tensor-core consumer for an FP8 (E4M3) cache and 16-bit q/out, G in {4, 8}.
+// E4M3 converts exactly to fp16, so both products run as fp16 mma.m16n8k16
+// (q is rounded to fp16 when it is bf16).  Fragment layout as in
+// MmaConsumer, with 16 dims per 16-byte chunk of a cache row:
+//   QK step (j, hf): k-slots (2c, 2c+1) <-> dims 16(4j+c) + 4hf + {0,1},
+//                    k-slots (2c+8, 2c+9) <-> dims 16(4j+c) + 4hf + {2,3};
+//   PV tile m: row r <-> dim r*D/8 + 2m, row r+8 <-> dim r*D/8 + 2m + 1;
+// V^T pairs of adjacent tokens are gathered byte-wise with permutes, then
+// converted pairwise.  The per-tensor scales enter the logits (k_scale) and
+// the output (v_scale).
+// ===========================================================================
+template <typename TQ, int D, int BS, int G>
+struct MmaConsumerFp8 {
+    using S = DecodeShape<TQ, fp8e4m3, D, BS, G>;
+    static_assert(sizeof(TQ) == 2, "q must be 16-bit");
+    static_assert(G <= 8, "the 8 MMA columns hold the query heads of one group");
+    static_assert(D % 64 == 0, "head_size 64 or 128");
+    static constexpr int KJ = D / 64;      // 16-dim chunks per lane per K row
+    static constexpr int MT = D / 16;      // PV MMAs
+    static constexpr int VB = D / 8;       // V bytes (dims) per lane per row
+
+    int r, c;
+    uint32_t qf[KJ][8];                    // fp16 pairs: [hf][b0, b1] for hf = 0..3
+    float o[MT][4];
+    float m0, m1, l0, l1;
+
+    __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+        uint32_t d;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+        return d;
+    }
+    __device__ __forceinline__ static uint32_t to_f16x2(uint32_t w) {
+        if constexpr (std::is_same<TQ, __half>::value) {
+            return w;
+        } else {
+            float lo, hi;
+            Elem<__nv_bfloat16>::widen2(w, lo, hi);
+            return Elem<__half>::pack2(lo, hi);
+        }
+    }
+    __device__ __forceinline__ static float lo_f(uint32_t w) {
+        return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+    }
+    __device__ __forceinline__ static float hi_f(uint32_t w) {
+        return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    }
+
+    __device__ __forceinline__ void init(int lane) {
+        r = lane >> 2;
+        c = lane & 3;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KJ; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qf[j][i] = 0u;
+    }
+
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float) {
+#pragma unroll
+        for (int j = 0; j < KJ; ++j) {
+            uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+            if (r < G) {
+                const uint4* qrow = reinterpret_cast<const uint4*>(qslot + r * S::QROW);
+                a = qrow[2 * (4 * j + c)];          // dims 16(4j+c) + 0..7
+                b = qrow[2 * (4 * j + c) + 1];      // dims 16(4j+c) + 8..15
+            }
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qf[j][i] = to_f16x2(w[i]);
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void slice(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float scale_log2) {
+        const uint4* k0 = reinterpret_cast<const uint4*>(Kt + r * S::ROW);
+        const uint4* k8 = reinterpret_cast<const uint4*>(Kt + (r + 8) * S::ROW);
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < KJ; ++j) {
+            const uint4 a = k0[4 * j + c];
+            const uint4 b = k8[4 * j + c];
+            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int hf = 0; hf < 4; ++hf)
+                mma(sc, e4m3x2_to_f16x2((uint16_t)(wa[hf] & 0xffffu)),
+                    e4m3x2_to_f16x2((uint16_t)(wb[hf] & 0xffffu)),
+                    e4m3x2_to_f16x2((uint16_t)(wa[hf] >> 16)), e4m3x2_to_f16x2((uint16_t)(wb[hf] >> 16)),
+                    qf[j][2 * hf], qf[j][2 * hf + 1]);
+        }
+        const bool v0 = r < nvalid, v8 = r + 8 < nvalid;
+        const float z0 = v0 ? sc[0] * scale_log2 : -INFINITY;
+        const float z1 = v0 ? sc[1] * scale_log2 : -INFINITY;
+        const float z2 = v8 ? sc[2] * scale_log2 : -INFINITY;
+        const float z3 = v8 ? sc[3] * scale_log2 : -INFINITY;
+        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float al0 = ex2(m0 - n0), al1 = ex2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const uint32_t pk_lo = Elem<__half>::pack2(ex2(z0 - n0), ex2(z1 - n1));
+        const uint32_t pk_hi = Elem<__half>::pack2(ex2(z2 - n0), ex2(z3 - n1));
+        l0 = l0 * al0 + lo_f(pk_lo) + lo_f(pk_hi);
+        l1 = l1 * al1 + hi_f(pk_lo) + hi_f(pk_hi);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            o[m][0] *= al0;
+            o[m][2] *= al0;
+            o[m][1] *= al1;
+            o[m][3] *= al1;
+        }
+        const int src0 = (2 * c) * 4 + (r >> 1), src1 = src0 + 4;
+        const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+        const uint32_t x0 = __shfl_sync(kFull, pk_lo, src0), x1 = __shfl_sync(kFull, pk_lo, src1);
+        const uint32_t y0 = __shfl_sync(kFull, pk_hi, src0), y1 = __shfl_sync(kFull, pk_hi, src1);
+        const uint32_t pb0 = prmt(x0, x1, sel), pb1 = prmt(y0, y1, sel);
+        // V rows 2c, 2c+1, 2c+8, 2c+9: bytes = dims r*D/8 .. +D/8
+        uint32_t w[4][VB / 4];
+        const int rows[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool ok = rows[i] < nvalid;       // masked tokens may hold NaN codes
+            const unsigned char* vr = Vt + rows[i] * S::ROW + r * VB;
+            if constexpr (VB == 16) {
+                uint4 v = *reinterpret_cast<const uint4*>(vr);
+                if (!ok) v = make_uint4(0u, 0u, 0u, 0u);
+                w[i][0] = v.x; w[i][1] = v.y; w[i][2] = v.z; w[i][3] = v.w;
+            } else {
+                uint2 v = *reinterpret_cast<const uint2*>(vr);
+                if (!ok) v = make_uint2(0u, 0u);
+                w[i][0] = v.x; w[i][1] = v.y;
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            // bytes 2m, 2m+1 of two rows: {A[2m], B[2m], A[2m+1], B[2m+1]}
+            const int wi = m >> 1;
+            const uint32_t sel2 = (m & 1) ? 0x7362u : 0x5140u;
+            const uint32_t lo = prmt(w[0][wi], w[1][wi], sel2);
+            const uint32_t hi = prmt(w[2][wi], w[3][wi], sel2);
+            mma(o[m], e4m3x2_to_f16x2((uint16_t)(lo & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo >> 16)),
+                e4m3x2_to_f16x2((uint16_t)(hi & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi >> 16)), pb0, pb1);
+        }
+    }
+
+    __device__ __forceinline__ void block(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float scale_log2) {
+#pragma unroll
+        for (int sl = 0; sl < BS / 16; ++sl) {
+            const int nv = nvalid - 16 * sl;
+            if (nv <= 0) break;
+            slice(Kt + sl * 16 * S::ROW, Vt + sl * 16 * S::ROW, nv, scale_log2);
+        }
+    }
+
+    __device__ __forceinline__ void finish(const StageMeta& mt, const DecodeParams& p) {
+        float t0 = l0, t1 = l1;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            t0 += __shfl_xor_sync(kFull, t0, off);
+            t1 += __shfl_xor_sync(kFull, t1, off);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int head = 2 * c + e;
+            if (head >= G) continue;
+            const float lt = e ? t1 : t0;
+            if (mt.flags & kWhole) {
+                const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
+                uint32_t words[MT];
+#pragma unroll
+                for (int m = 0; m < MT; ++m) words[m] = Elem<TQ>::pack2(o[m][e] * inv, o[m][2 + e] * inv);
+                uint4* orow = reinterpret_cast<uint4*>(
+                    reinterpret_cast<TQ*>(p.out) +
+                    ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + head) * D + r * (D / 8));
+#pragma unroll
+                for (int ch = 0; ch < MT / 4; ++ch)
+                    orow[ch] = make_uint4(words[4 * ch], words[4 * ch + 1], words[4 * ch + 2],
+                                          words[4 * ch + 3]);
+            } else {
+                const float vs = p.v_scale;
+                float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + head) * D +
+                                                         r * (D / 8));
+#pragma unroll
+                for (int m = 0; m < MT; m += 2)
+                    prow[m / 2] = make_float4(o[m][e] * vs, o[m][2 + e] * vs, o[m + 1][e] * vs,
+                                              o[m + 1][2 + e] * vs);
+                if (r == 0)
+                    p.part_ml[(size_t)mt.item * G + head] = make_float2(e ? m1 : m0, lt);
+            }
+        }
+    }
 };
 
-template <typename T, int D, int BS, int G>
-using ConsumerFor = typename std::conditional<UseMma<T, G>::value, MmaConsumer<T, D, BS, G>,
-                                              FmaConsumer<T, D, BS, G>>::type;
+// Tensor cores where the fp32 FMA path is issue-bound: groups of 4-8 query
+// heads over a 16-bit cache, and every group over an FP8 cache (half the
+// bytes per element, so twice the FMA work per byte); columns of the 8-wide
+// MMA beyond G are zero padding.
+template <typename TQ, typename TC, int G>
+struct UseMma {
+    static constexpr bool value =
+        sizeof(TQ) == 2 && ((std::is_same<TQ, TC>::value && (G == 4 || G == 8)) ||
+                            (std::is_same<TC, fp8e4m3>::value && G <= 8));
+};
+
+template <typename TQ, typename TC, int D, int BS, int G>
+using ConsumerFor = typename std::conditional<
+    UseMma<TQ, TC, G>::value,
+    typename std::conditional<std::is_same<TC, fp8e4m3>::value, MmaConsumerFp8<TQ, D, BS, G>,
+                              MmaConsumer<TQ, D, BS, G>>::type,
+    FmaConsumer<TQ, TC, D, BS, G>>::type;
 
 // ===========================================================================
 // Partition size for the call, chosen identically by every CTA.  With NW
@@ -526,10 +762,11 @@ __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, cons
 // ===========================================================================
 // The kernel: prologue, producer (bulk-copy ring) and consumer loop.
 // ===========================================================================
-template <typename T, int D, int BS, int G>
+template <typename TQ, typename TC, int D, int BS, int G>
 __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams p) {
-    using S = DecodeShape<T, D, BS, G>;
-    using L = WarpSmem<T, D, BS, G>;
+    using S = DecodeShape<TQ, TC, D, BS, G>;
+    using L = WarpSmem<TQ, TC, D, BS, G>;
+    constexpr bool kSameType = std::is_same<TQ, TC>::value;   // fused cache write needs it
     extern __shared__ __align__(128) unsigned char smem[];
 
     const int nseq = p.num_seqs;
@@ -610,7 +847,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         it.nblk = max(used, 1);
         if (lane < used)
             it.tbl = __ldg(p.block_tables + (size_t)lo * p.max_blocks_per_seq + it.tok0 / BS + lane);
-        if (p.slot_mapping != nullptr && it.ntok > 0 && it.tok0 + it.ntok == s_len[lo])
+        if (kSameType && p.slot_mapping != nullptr && it.ntok > 0 && it.tok0 + it.ntok == s_len[lo])
             it.slot = __ldg(p.slot_mapping + lo);
         return it;
     };
@@ -630,9 +867,9 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
     int issue_st = 0;
     int issued = 0;
     const size_t tile_elems = (size_t)BS * D;
-    const T* kc = reinterpret_cast<const T*>(p.k_cache);
-    const T* vc = reinterpret_cast<const T*>(p.v_cache);
-    const T* qg = reinterpret_cast<const T*>(p.q);
+    const TC* kc = reinterpret_cast<const TC*>(p.k_cache);
+    const TC* vc = reinterpret_cast<const TC*>(p.v_cache);
+    const TQ* qg = reinterpret_cast<const TQ*>(p.q);
 
     auto issue = [&]() {
         if (P.idx >= n_items) return;
@@ -664,8 +901,8 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
                                    (newrow >= 0 ? 2 * S::ROW : 0);
             mbar_arrive_expect_tx(bar, bytes);
             if (newrow >= 0) {
-                const T* kn = reinterpret_cast<const T*>(p.key) + (size_t)P.s * p.key_stride + (size_t)P.g * D;
-                const T* vn = reinterpret_cast<const T*>(p.value) + (size_t)P.s * p.value_stride + (size_t)P.g * D;
+                const TC* kn = reinterpret_cast<const TC*>(p.key) + (size_t)P.s * p.key_stride + (size_t)P.g * D;
+                const TC* vn = reinterpret_cast<const TC*>(p.value) + (size_t)P.s * p.value_stride + (size_t)P.g * D;
                 bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW), kn, S::ROW, bar);
                 bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW + S::ROW), vn, S::ROW, bar);
             }
@@ -693,7 +930,8 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
     };
 
     // ---- consumer ----
-    ConsumerFor<T, D, BS, G> cons;
+    ConsumerFor<TQ, TC, D, BS, G> cons;
+    const float qscale = p.scale_log2 * p.k_scale;   // logits in log2 units, cache scale folded in
     cons.init(lane);
 
     for (int i = 0; i < R; ++i) issue();
@@ -710,7 +948,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
             break;
         }
         const StageMeta mt = meta[cons_st];
-        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, p.scale_log2);
+        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, qscale);
         if (mt.newrow >= 0) {
             // Fused cache write: put the new token's K and V rows into the tile
             // (it holds the slot's old bytes) and into the cache slot.
@@ -723,7 +961,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
                 const int c16 = ch - v * (S::ROW / 16);
                 const uint4 w = reinterpret_cast<const uint4*>(nb + v * S::ROW)[c16];
                 reinterpret_cast<uint4*>(Kt + v * S::TILE + mt.newrow * S::ROW)[c16] = w;
-                T* cache = const_cast<T*>(v ? vc : kc);
+                TC* cache = const_cast<TC*>(v ? vc : kc);
                 reinterpret_cast<uint4*>(cache + slot_off)[c16] = w;
             }
             fence_proxy_async();     // these generic writes precede the stage's next bulk copy
@@ -731,7 +969,7 @@ __global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams
         }
         if (mt.nvalid > 0) {
             const unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
-            cons.block(Kt, Kt + S::TILE, mt.nvalid, p.scale_log2);
+            cons.block(Kt, Kt + S::TILE, mt.nvalid, qscale);
         }
         if (mt.flags & kLast) cons.finish(mt, p);
         __syncwarp();

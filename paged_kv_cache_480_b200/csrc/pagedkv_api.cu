@@ -108,7 +108,14 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, 
     return w;
 }
 
-uint32_t warp_smem(pkv_dtype t, int D, int BS, int G, int R) {
+uint32_t warp_smem(pkv_dtype t, bool fp8_cache, int D, int BS, int G, int R) {
+    if (fp8_cache) {
+        switch (t) {
+            case PKV_F32: return pkv::warp_smem_f32_fp8(D, BS, G, R);
+            case PKV_F16: return pkv::warp_smem_f16_fp8(D, BS, G, R);
+            default: return pkv::warp_smem_bf16_fp8(D, BS, G, R);
+        }
+    }
     switch (t) {
         case PKV_F32: return pkv::warp_smem_f32(D, BS, G, R);
         case PKV_F16: return pkv::warp_smem_f16(D, BS, G, R);
@@ -179,7 +186,8 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
                        int num_kv_heads, int block_size, int num_seqs, int num_heads,
                        int head_size, int num_blocks, int max_blocks_per_seq, int max_context_len,
                        pkv_dtype dtype, int partition_size, void* workspace,
-                       size_t workspace_bytes, void* stream, const AppendArgs* app) {
+                       size_t workspace_bytes, void* stream, const AppendArgs* app,
+                       bool fp8_cache = false, float k_scale = 1.f, float v_scale = 1.f) {
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return PKV_ERR_INVALID_ARG;
     pkv_status st = check_shape(num_seqs, num_heads, num_kv_heads, head_size, block_size,
@@ -190,7 +198,7 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned4(block_tables) || !aligned4(context_lens))
         return PKV_ERR_INVALID_ARG;
-    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (!(scale == scale) || !(k_scale > 0.f) || !(v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
     int ps_hi = 0;
     const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
                                      partition_size, &ps_hi);
@@ -207,18 +215,22 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     // Shared memory: per-CTA lengths and prefix sums, then one ring per warp.
     const uint32_t seq_smem = (uint32_t)round_up(sizeof(int32_t) * (2 * (size_t)num_seqs + 1), 128);
     // Eight consumer warps per SM hide the per-block latency of the consumer
-    // math (measured: six warps lose 10%, ten or twelve gain nothing); a
-    // ring of two stages per warp then keeps enough bytes in flight.  Use
-    // the deepest ring (up to 4) that still fits eight warps, else fewer
-    // warps with two stages.
+    // math for 16-bit caches (measured: six warps lose 10%, ten or twelve
+    // gain nothing); a ring of two stages per warp then keeps enough bytes
+    // in flight.  Use the deepest ring (up to 4) that still fits eight
+    // warps, else fewer warps with two stages.
     int R = 4;
-    uint32_t per_warp = warp_smem(dtype, head_size, block_size, G, R);
+    uint32_t per_warp = warp_smem(dtype, fp8_cache, head_size, block_size, G, R);
     while (R > 2 && (pkv::kMaxDynSmem - seq_smem) / per_warp < 8) {
         --R;
-        per_warp = warp_smem(dtype, head_size, block_size, G, R);
+        per_warp = warp_smem(dtype, fp8_cache, head_size, block_size, G, R);
     }
     int W = (int)((pkv::kMaxDynSmem - seq_smem) / per_warp);
-    if (W > 8) W = 8;
+    // An FP8 cache halves the bytes per element, so each warp must retire
+    // blocks twice as fast: give it up to 12 consumer warps (measured: 8 -> 12
+    // warps is 1.25x; the 16-bit path gains nothing past 8).
+    const int w_cap = fp8_cache ? 12 : 8;
+    if (W > w_cap) W = w_cap;
     if (W < 1) return PKV_ERR_UNSUPPORTED;
 
     unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -235,6 +247,8 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     p.prefix_out = reinterpret_cast<int32_t*>(ws + wl.prefix);
     p.errors = errors;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.num_seqs = num_seqs;
     p.num_heads = num_heads;
     p.num_kv_heads = num_kv_heads;
@@ -262,10 +276,19 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     const size_t smem = seq_smem + (size_t)W * per_warp;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    switch (dtype) {
-        case PKV_F32: e = pkv::decode_f32(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
-        case PKV_F16: e = pkv::decode_f16(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
-        default: e = pkv::decode_bf16(p, head_size, block_size, G, dim3(ctas), dim3(32 * W), smem, s); break;
+    const dim3 grid(ctas), block(32 * W);
+    if (fp8_cache) {
+        switch (dtype) {
+            case PKV_F32: e = pkv::decode_f32_fp8(p, head_size, block_size, G, grid, block, smem, s); break;
+            case PKV_F16: e = pkv::decode_f16_fp8(p, head_size, block_size, G, grid, block, smem, s); break;
+            default: e = pkv::decode_bf16_fp8(p, head_size, block_size, G, grid, block, smem, s); break;
+        }
+    } else {
+        switch (dtype) {
+            case PKV_F32: e = pkv::decode_f32(p, head_size, block_size, G, grid, block, smem, s); break;
+            case PKV_F16: e = pkv::decode_f16(p, head_size, block_size, G, grid, block, smem, s); break;
+            default: e = pkv::decode_bf16(p, head_size, block_size, G, grid, block, smem, s); break;
+        }
     }
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (wl.max_parts > 1) {
@@ -303,6 +326,20 @@ pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                        block_size, num_seqs, num_heads, head_size, num_blocks, max_blocks_per_seq,
                        max_context_len, dtype, partition_size, workspace, workspace_bytes, stream,
                        nullptr);
+}
+
+pkv_status paged_attention_decode_fp8kv(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const int32_t* block_tables,
+                                        const int32_t* context_lens, float scale, float k_scale,
+                                        float v_scale, int num_kv_heads, int block_size,
+                                        int num_seqs, int num_heads, int head_size, int num_blocks,
+                                        int max_blocks_per_seq, int max_context_len,
+                                        pkv_dtype dtype, int partition_size, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                       block_size, num_seqs, num_heads, head_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, dtype, partition_size, workspace, workspace_bytes, stream,
+                       nullptr, true, k_scale, v_scale);
 }
 
 pkv_status paged_attention_decode_append(void* out, const void* q, const void* key,
@@ -369,6 +406,52 @@ pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, 
     p.block_size = block_size;
     p.num_blocks = num_blocks;
     if (pkv::launch_reshape_and_cache(p, sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+pkv_status reshape_and_cache_fp8kv(const void* key, const void* value, void* k_cache,
+                                  void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                  int num_kv_heads, int head_size, int block_size, int num_blocks,
+                                  int64_t key_token_stride, int64_t value_token_stride,
+                                  pkv_dtype dtype, float k_scale, float v_scale, void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (head_size != 64 && head_size != 128) return PKV_ERR_UNSUPPORTED;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    const int eb = elem_bytes(dtype);
+    if (key_token_stride < (int64_t)num_kv_heads * head_size ||
+        value_token_stride < (int64_t)num_kv_heads * head_size ||
+        (key_token_stride * eb) % 16 || (value_token_stride * eb) % 16)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PKV_ERR_INVALID_ARG;
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    pkv_status st = device_info(&sms, &errors);
+    if (st != PKV_OK) return st;
+    pkv::CacheWriteFp8Params p;
+    p.key = key;
+    p.value = value;
+    p.k_cache = static_cast<unsigned char*>(k_cache);
+    p.v_cache = static_cast<unsigned char*>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.errors = errors;
+    p.key_stride = key_token_stride;
+    p.value_stride = value_token_stride;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.head_size = head_size;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    p.src_dtype = dtype;
+    if (pkv::launch_reshape_and_cache_fp8(p, sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return PKV_ERR_CUDA;
     return PKV_OK;
 }

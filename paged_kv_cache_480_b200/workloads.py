@@ -259,6 +259,24 @@ def make_tensors(layout, device="cpu", pending_new_token=True):
     return dict(q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new, v_new=v_new)
 
 
+def make_tensors_fp8(layout, device="cpu", k_scale=1.0 / 64, v_scale=1.0 / 64, pending_new_token=True):
+    """Tensors for an FP8 E4M3 cache: q, k_new, v_new in the layout's dtype;
+    k_cache / v_cache uint8 codes of the same N(0,1) draws divided by the
+    scales (rounded by torch's float8_e4m3fn cast, values well inside the
+    finite range); slots without a context token hold the NaN code 0x7f."""
+    import torch
+    ten = make_tensors(layout, device=device, pending_new_token=pending_new_token)
+    out = dict(q=ten["q"], k_new=ten["k_new"], v_new=ten["v_new"])
+    for name, sc in (("k_cache", k_scale), ("v_cache", v_scale)):
+        x = ten[name].float()
+        nan = torch.isnan(x)
+        codes = (x.nan_to_num(0.0) / sc).to(torch.float8_e4m3fn).view(torch.uint8)
+        codes[nan] = 0x7f
+        out[name] = codes
+        del x
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Parallel sampling with copy-on-write (cow_bf16).
 # ---------------------------------------------------------------------------
