@@ -46,6 +46,7 @@ def _load():
         lib.orc_copy_blocks.argtypes = [P, I, P, I, I64]
         lib.orc_swap_blocks.argtypes = [P, P, I, P, I, I64]
         lib.orc_round.argtypes = [P, P, I, I64]
+        lib.orc_paged_prefill.argtypes = [P, P, P, P, I, P, I, P, P, I, I, I, I, I, D, I]
         lib.orc_paged_attention_ex.argtypes = [P, P, I, P, P, I, D, D, P, I, P, I, I, I, I, I, D, I]
         lib.orc_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.orc_e4m3_to_double.restype = D
@@ -259,3 +260,22 @@ def reshape_and_cache_fp8(k, v, src_dtype, k_cache, v_cache, slot_mapping, block
     _load().orc_reshape_and_cache_e4m3(_ptr(k), _ptr(v), sc, _ptr(k_cache), _ptr(v_cache), _ptr(sm),
                                        T, Hkv, D, block_size, Hkv * D, Hkv * D,
                                        ctypes.c_float(k_scale), ctypes.c_float(v_scale))
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale, dtype,
+                  num_kv_heads, block_size, nthreads=None):
+    """fp64 causal prefill attention: q [T, H, D] packed by sequence
+    (query_start_loc int32 [S+1]); the last n_s tokens of each sequence's
+    context are its queries.  Returns [T, H, D] float64."""
+    code = DTYPE_CODES[dtype]
+    q, kc, vc = _raw(q, code), _raw(k_cache, code), _raw(v_cache, code)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    T, H, D = q.shape
+    assert qsl[-1] == T
+    out = np.zeros((T, H, D), np.float64)
+    _load().orc_paged_prefill(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), code, _ptr(bt), bt.shape[1],
+                              _ptr(cl), _ptr(qsl), len(cl), H, num_kv_heads, D, block_size,
+                              float(scale), nthreads or default_threads())
+    return out

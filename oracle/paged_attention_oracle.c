@@ -208,7 +208,7 @@ static void orc_gather(double* K, double* V, const void* k_cache, const void* v_
 static void orc_row(double* acc, double* m_out, double* l_out, double* weights,
                     const void* q, int qdtype, const void* k_cache, const void* v_cache, int cdtype,
                     double k_scale, double v_scale, const int32_t* table_row, int t0, int t1,
-                    int s, int h, int num_heads, int num_kv_heads, int head_size, int block_size,
+                    int64_t qrow, int h, int num_heads, int num_kv_heads, int head_size, int block_size,
                     double scale) {
     int G = num_heads / num_kv_heads;
     int kv_head = h / G;
@@ -225,7 +225,7 @@ static void orc_row(double* acc, double* m_out, double* l_out, double* weights,
     orc_gather(K, V, k_cache, v_cache, cdtype, k_scale, v_scale, table_row, t0, t1, kv_head,
                num_kv_heads, block_size, head_size);
     for (int d = 0; d < head_size; ++d)
-        qd[d] = orc_load(q, qdtype, ((int64_t)s * num_heads + h) * head_size + d);
+        qd[d] = orc_load(q, qdtype, (qrow * num_heads + h) * head_size + d);
 
     double m = -INFINITY;
     for (int t = 0; t < n; ++t) {
@@ -439,5 +439,40 @@ void orc_reshape_and_cache_e4m3(const void* k, const void* v, int src_dtype, uin
                 v_cache[dst] = orc_quantize_e4m3(
                     orc_load(v, src_dtype, (int64_t)i * value_stride + (int64_t)g * head_size + d), v_scale);
             }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Paged prefill / chunked-prefill attention [P1 workflow: prefill writes the
+ * input tokens' KV into pages and decoding continues from them; P1 usage:
+ * enable_chunked_prefill].  Sequence s holds context_lens[s] = L tokens in
+ * its blocks, the last n = qsl[s+1] - qsl[s] of which are this call's
+ * queries, packed as q rows qsl[s] .. qsl[s+1]-1.  Query i sits at position
+ * L - n + i and attends causally to keys 0 .. L - n + i:
+ *   out[qsl[s]+i, h, :] = sum_{t <= L-n+i} softmax_t(scale q.K_s[t]) V_s[t].
+ * q, out: [T][H][D] with T = qsl[S]; out in fp64.
+ * ------------------------------------------------------------------- */
+void orc_paged_prefill(double* out, const void* q, const void* k_cache, const void* v_cache,
+                       int dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                       const int32_t* context_lens, const int32_t* query_start_loc, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_size, int block_size, double scale,
+                       int nthreads) {
+    int64_t T = query_start_loc[num_seqs];
+    int64_t rows = T * num_heads;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 4)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t row = r / num_heads;
+        int h = (int)(r % num_heads);
+        int s = 0;
+        while (query_start_loc[s + 1] <= row) ++s;
+        int n = query_start_loc[s + 1] - query_start_loc[s];
+        int L = context_lens[s];
+        int pos = L - n + (int)(row - query_start_loc[s]);
+        double m, l;
+        double* o = out + r * head_size;
+        orc_row(o, &m, &l, NULL, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0,
+                block_tables + (int64_t)s * max_blocks_per_seq, 0, pos + 1, row, h, num_heads,
+                num_kv_heads, head_size, block_size, scale);
+        for (int d = 0; d < head_size; ++d) o[d] = (l > 0.0) ? o[d] / l : 0.0;
     }
 }

@@ -379,3 +379,49 @@ def test_swap_blocks_matches_fancy_indexing():
     oracle.swap_blocks(src, dst, mapping)
     for d, r in zip(dst, ref):
         assert np.array_equal(d, r)
+
+
+# ---------------------------------------------------------------------------
+# prefill / chunked prefill
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,H,Hkv,D,bs,lens,nq", [
+    ("bf16", 4, 4, 64, 16, [20, 37, 5], [20, 10, 1]),       # full prefill, a chunk, a decode step
+    ("f16", 8, 2, 128, 16, [70, 16, 33], [33, 16, 7]),
+    ("bf16", 8, 1, 64, 32, [100, 3], [64, 3]),
+])
+def test_prefill_matches_causal_sdpa(dtype, H, Hkv, D, bs, lens, nq):
+    rng = np.random.default_rng(30)
+    q_dec, Kc, Vc, kc, vc, _, tables = build_paged(rng, lens, H, Hkv, D, bs, dtype)
+    tdt = wl.torch_dtype(dtype)
+    qsl = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    qt = (torch.from_numpy(rng.standard_normal((int(qsl[-1]), H, D)))).to(tdt)
+    q_raw = _raw_from_torch(qt, dtype)
+    scale = 1.0 / math.sqrt(D)
+    got = oracle.paged_prefill(q_raw, kc, vc, tables, np.array(lens, np.int32), qsl, scale, dtype, Hkv, bs)
+    G = H // Hkv
+    for s, (L, n) in enumerate(zip(lens, nq)):
+        K = Kc[s].repeat_interleave(G, 0)
+        V = Vc[s].repeat_interleave(G, 0)
+        q = qt[qsl[s]:qsl[s + 1]].double().transpose(0, 1)            # [H, n, D]
+        # query i at position L - n + i sees keys 0 .. L - n + i
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(got[qsl[s]:qsl[s + 1]], ref.transpose(0, 1).numpy(), rtol=0, atol=1e-12)
+        if n == L:   # a whole prompt is the textbook causal attention
+            ref2 = torch.nn.functional.scaled_dot_product_attention(q, K, V, is_causal=True, scale=scale)
+            np.testing.assert_allclose(got[qsl[s]:qsl[s + 1]], ref2.transpose(0, 1).numpy(), atol=1e-12)
+
+
+def test_prefill_last_query_equals_decode():
+    """The last query of every sequence attends to the whole context: the decode definition."""
+    rng = np.random.default_rng(31)
+    lens, nq = [45, 16, 90], [5, 16, 1]
+    _, Kc, Vc, kc, vc, _, tables = build_paged(rng, lens, 4, 2, 64, 16, "bf16")
+    qsl = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    qt = torch.from_numpy(rng.standard_normal((int(qsl[-1]), 4, 64))).to(torch.bfloat16)
+    q_raw = _raw_from_torch(qt, "bf16")
+    L = np.array(lens, np.int32)
+    pre = oracle.paged_prefill(q_raw, kc, vc, tables, L, qsl, 0.125, "bf16", 2, 16)
+    last = q_raw[qsl[1:] - 1]
+    dec = oracle.paged_attention(last, kc, vc, tables, L, 0.125, "bf16", 2, 16)
+    assert np.array_equal(pre[qsl[1:] - 1], dec)
