@@ -42,8 +42,10 @@ def parse():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--measure", default="decode", choices=["decode", "swap"],
-                    help="swap: swap_blocks between the GPU pool and a pinned host pool")
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "prefill"],
+                    help="swap: swap_blocks between the GPU pool and a pinned host pool; "
+                         "prefill: cache write + causal prefill attention (--workload "
+                         "prefill_llama7b_bf16 or chunked_gqa_bf16)")
     ap.add_argument("--kv-cache", default="auto", choices=["auto", "fp8"],
                     help="fp8: E4M3 cache written by reshape_and_cache_fp8kv, read by the fp8 decode")
     ap.add_argument("--fused", action="store_true",
@@ -58,6 +60,20 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def tensor_peak():
+    """Dense bf16 tensor throughput (TFLOP/s) measured by cuBLAS as a burst."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 # ---------------------------------------------------------------------------
@@ -559,6 +575,268 @@ def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
     return result
 
 
+# ---------------------------------------------------------------------------
+# prefill: cache write of the chunk's K/V + causal prefill attention
+# ---------------------------------------------------------------------------
+PREFILL_METRIC = "paged prefill attn: achieved TFLOP/s (causal pairs x 4 x head_size x heads)"
+
+
+def prefill_flops(lay):
+    from paged_kv_cache_480_b200 import workloads as wl
+    return 4 * lay.head_size * lay.num_heads * wl.prefill_pairs(lay)
+
+
+def prefill_slots(lay):
+    """Cache slots of every sequence's query tokens (positions L - n .. L - 1)."""
+    bs = lay.block_size
+    out = []
+    for s, (L, n) in enumerate(zip(lay.context_lens, lay.extra["query_lens"])):
+        pos = np.arange(int(L) - int(n), int(L))
+        out.append(lay.block_tables[s, pos // bs].astype(np.int64) * bs + pos % bs)
+    return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+
+def prefill_workload(name, device):
+    from paged_kv_cache_480_b200 import workloads as wl
+    if name not in wl.PREFILL_CONFIGS:
+        name = "prefill_llama7b_bf16"
+    lay = wl.make_prefill_layout(name)
+    ten = wl.make_prefill_tensors(lay, device=device)
+    slots = prefill_slots(lay)
+    # the chunk's own K/V as the step writes them: the values already at those
+    # slots, so repeated steps leave the cache unchanged
+    sl = torch_from(slots, device)
+    nb, hkv, bs, d = ten["k_cache"].shape
+    flat_k = ten["k_cache"].permute(0, 2, 1, 3).reshape(nb * bs, hkv, d)
+    flat_v = ten["v_cache"].permute(0, 2, 1, 3).reshape(nb * bs, hkv, d)
+    ten["k_new"] = flat_k[sl].contiguous()
+    ten["v_new"] = flat_v[sl].contiguous()
+    ten["slots"] = sl
+    return lay, ten
+
+
+def torch_from(a, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def prefill_oracle_sample(lay, host, budget_s, nseq):
+    """Oracle prefill over the first nseq sequences (all heads), repeated to
+    ~budget_s; returns (TFLOP/s, seconds, flops, passes, threads)."""
+    import oracle
+    from paged_kv_cache_480_b200 import workloads as wl
+    qsl = lay.extra["query_start_loc"]
+    sub = wl.Layout(**{**lay.__dict__, "num_seqs": nseq, "context_lens": lay.context_lens[:nseq],
+                       "block_tables": lay.block_tables[:nseq], "slot_mapping": lay.slot_mapping[:nseq],
+                       "extra": {"query_lens": lay.extra["query_lens"][:nseq],
+                                 "query_start_loc": qsl[:nseq + 1]}})
+    flops = prefill_flops(sub)
+    threads = oracle.default_threads()
+    q = host["q"][:int(qsl[nseq])]
+    total_t, reps = 0.0, 0
+    while total_t < budget_s or reps == 0:
+        t0 = time.perf_counter()
+        oracle.paged_prefill(q, host["k_cache"], host["v_cache"], sub.block_tables, sub.context_lens,
+                             qsl[:nseq + 1], lay.scale, lay.dtype, lay.num_kv_heads, lay.block_size,
+                             nthreads=threads)
+        total_t += time.perf_counter() - t0
+        reps += 1
+    return flops * reps / total_t / 1e12, total_t, flops * reps, reps, threads
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    pkv.load_library()
+    lay, ten = prefill_workload(args.workload, device)
+    bt = torch_from(lay.block_tables, device)
+    cl = torch_from(lay.context_lens, device)
+    qsl = torch_from(lay.extra["query_start_loc"], device)
+    mq = int(lay.extra["query_lens"].max())
+    T = int(lay.extra["query_start_loc"][-1])
+    out = torch.empty_like(ten["q"])
+    stream = torch.cuda.current_stream(device)
+    ev = []
+
+    def step(record=False):
+        pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], ten["slots"],
+                              stream=stream)
+        if record:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        pkv.paged_attention_prefill(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, qsl, lay.scale,
+                                    max_query_len=mq, stream=stream)
+        if record:
+            b.record(stream)
+            ev.append((a, b))
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    assert pkv.read_device_errors() == 0
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.05)
+        torch.cuda.synchronize(device)
+        clk.mark_start()
+        start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        clk.mark_end()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ms_total = max_over_ranks(start.elapsed_time(end), world, device)
+    errors = pkv.read_device_errors()
+    flops = prefill_flops(lay)
+    ms_step = ms_total / args.steps
+    if rank != 0:
+        return None
+    peak, peak_kind = tensor_peak()
+    k_ms = [a.elapsed_time(b) for a, b in ev]
+    k_avg = sum(k_ms) / len(k_ms)
+    achieved = flops / (k_avg * 1e-3) / 1e12
+    kv_bytes = lay.kv_bytes()
+    result = {"metric": PREFILL_METRIC, "value": world * flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+              "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+              "tokens_per_s": world * T / (ms_step * 1e-3), "higher_is_better": True, "scaling": "weak",
+              "vs_baseline": None, "dtype": lay.dtype, "data": "synthetic",
+              "config": {"workload": lay.name, "num_seqs": lay.num_seqs, "query_tokens": T,
+                         "num_heads": lay.num_heads, "num_kv_heads": lay.num_kv_heads,
+                         "head_size": lay.head_size, "block_size": lay.block_size,
+                         "num_blocks": lay.num_blocks, "max_context_len": lay.max_context_len,
+                         "max_query_len": mq, "causal_pairs": int(flops // (4 * lay.head_size * lay.num_heads)),
+                         "flops_per_step": flops,
+                         "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V in the cache",
+                         "parallelism": f"replicas x{world}"},
+              "roofline": {"kernel": "paged_attention_prefill", "bound": "tensor", "achieved": achieved,
+                           "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                           "traffic": None, "algorithmic_flops": flops, "avg_call_us": k_avg * 1e3},
+              "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "device_errors": errors}
+    if not args.no_e2e:
+        result["e2e"] = run_prefill_e2e(args, lay, ten, device, flops)
+    if not args.no_cpu_baseline and world == 1:
+        host = host_arrays(ten, lay.dtype)
+        tf, t, f, reps, threads = prefill_oracle_sample(lay, host, 10.0, 1)
+        result["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                  "sample": f"fp64 oracle prefill of the first sequence (all heads), "
+                                            f"{reps} passes in {t:.1f} s"}
+    return result
+
+
+def run_prefill_e2e(args, lay, ten, device, flops):
+    """The prefill step through the C ABI with its inputs (q, the chunk's
+    K/V, slots, tables, lengths, query offsets) in pinned host memory, one
+    copy in and the output out every step; a CUDA graph of the step replayed."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    parts = [("q", ten["q"]), ("k", ten["k_new"]), ("v", ten["v_new"]), ("sm", ten["slots"]),
+             ("bt", torch.from_numpy(lay.block_tables)), ("cl", torch.from_numpy(lay.context_lens)),
+             ("qsl", torch.from_numpy(lay.extra["query_start_loc"]))]
+    offs, total = {}, 0
+    for name, t in parts:
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(total, dtype=torch.uint8, device=device)
+
+    def view(buf, name, t):
+        n = t.numel() * t.element_size()
+        return buf[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+
+    for name, t in parts:
+        view(h_buf, name, t).copy_(t.detach().cpu())
+    d = {name: view(d_buf, name, t) for name, t in parts}
+    out = torch.empty_like(ten["q"])
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    mq = int(lay.extra["query_lens"].max())
+    h2d = sum(t.numel() * t.element_size() for _, t in parts)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def body(stream):
+        d_buf.copy_(h_buf, non_blocking=True)
+        pkv.reshape_and_cache(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], stream=stream)
+        pkv.paged_attention_prefill(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"], d["qsl"],
+                                    lay.scale, max_query_len=mq, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    n_steps = max(args.steps, 50)
+
+    def timed(run, sync):
+        for _ in range(3):
+            run()
+            sync()
+        times = []
+        for _ in range(n_steps):
+            t0 = time.perf_counter()
+            run()
+            sync()
+            times.append(time.perf_counter() - t0)
+        return statistics.median(times)
+
+    stream = torch.cuda.current_stream(device)
+    eager = timed(lambda: body(stream), stream.synchronize)
+    result = {"value": flops / eager / 1e12, "unit": "TFLOP/s", "us_per_step": eager * 1e6,
+              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager",
+              "timing": f"median of {n_steps} wall-clock steps, each ending in a host sync"}
+    try:
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            body(cap)
+            cap.synchronize()
+            with torch.cuda.graph(graph, stream=cap):
+                body(cap)
+        stream.wait_stream(cap)
+        replay = timed(graph.replay, torch.cuda.synchronize)
+        assert pkv.read_device_errors() == 0
+        result.update({"value": flops / replay / 1e12, "us_per_step": replay * 1e6,
+                       "mode": "cuda graph of the step, replayed per step",
+                       "eager_value": flops / eager / 1e12, "eager_us_per_step": eager * 1e6})
+        del graph
+    except Exception as e:
+        result["graph_error"] = str(e)[:200]
+    return result
+
+
+def run_prefill_reference(args, rank, world):
+    """The oracle prefill, as it stands, on this host's cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    from paged_kv_cache_480_b200 import workloads as wl
+    name = args.workload if args.workload in wl.PREFILL_CONFIGS else "prefill_llama7b_bf16"
+    lay = wl.make_prefill_layout(name)
+    ten = wl.make_prefill_tensors(lay, device="cpu")
+    host = host_arrays(ten, lay.dtype)
+    for _ in range(args.warmup):
+        prefill_oracle_sample(lay, host, 0.0, 1)
+    times, flops = [], 0
+    for _ in range(args.steps):
+        tf, t, f, reps, threads = prefill_oracle_sample(lay, host, 0.0, 1)
+        times.append(t)
+        flops = f
+    avg = sum(times) / len(times)
+    value = flops / avg / 1e12
+    sample = "the first sequence of the workload (all heads) per step"
+    return {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": avg * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": name, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def run_swap(args, rank, world, local_rank):
     """swap_blocks throughput, device <-> pinned host, against a contiguous
     pinned copy of the same size measured in the same run (the host link's
@@ -623,7 +901,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        res = run_reference(args, rank, world)
+        res = run_prefill_reference(args, rank, world) if args.measure == "prefill" else \
+            run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
         return
@@ -640,7 +919,10 @@ def main():
                 if rank == 0:
                     print(json.dumps(line), flush=True)
             return
-        res = run_ours(args, rank, world, local_rank)
+        if args.measure == "prefill":
+            res = run_prefill(args, rank, world, local_rank)
+        else:
+            res = run_ours(args, rank, world, local_rank)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

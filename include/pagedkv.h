@@ -318,6 +318,52 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
 /* Synchronise the stream, return the sticky device-check bits of the
  * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
  * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */
+/* ---------------------------------------------------------------------------
+ * paged_attention_prefill -- causal attention of a batch of prompts, or of
+ * prompt chunks, whose keys and values are already in the paged cache.
+ *
+ * Defines: sequence s has L = context_lens[s] tokens in its blocks and n =
+ * query_start_loc[s+1] - query_start_loc[s] queries, the last n of those
+ * tokens.  For query i (row query_start_loc[s] + i of q) at position
+ * p = L - n + i,
+ *   out[row, h, :] = sum_{t <= p} softmax_t(scale * q[row,h] . K_s[t]) V_s[t]
+ * with K_s / V_s read through the block table as in the decode call.  The
+ * pages' serving workflow ("PyTorch-CUDA-v2.9 image enables PagedAttention",
+ * workflow list, and its chunked-prefill usage notes): the prompt's keys and
+ * values are first written into pages (reshape_and_cache), then attended
+ * causally; a chunk of a long prompt attends to every earlier chunk's keys
+ * already in the pages plus its own.  n == L is a whole prompt; n == 1 is a
+ * decode step.
+ *
+ *   out            device, [num_tokens][num_heads][head_size], dtype (written;
+ *                  rows of every sequence's queries)
+ *   q              device, [num_tokens][num_heads][head_size], dtype
+ *   k_cache, v_cache, block_tables   as in paged_attention_decode
+ *   context_lens   device, int32 [num_seqs]: tokens in the cache for s,
+ *                  including this call's queries (written beforehand)
+ *   query_start_loc device, int32 [num_seqs + 1], non-decreasing,
+ *                  query_start_loc[0] = 0, query_start_loc[num_seqs] = num_tokens
+ *   max_query_len  host-known bound of n over the batch (> 0 unless
+ *                  num_tokens == 0); sizes the grid
+ *   dtype          f16 or bf16 (q, caches and out the same); the products
+ *                  run on the tensor cores with fp32 accumulation and the
+ *                  softmax weights rounded to dtype before the product with V
+ *
+ * Device checks: n < 0, n > L, n > max_query_len, L > max_blocks_per_seq *
+ * block_size or queries outside [0, num_tokens) set PKV_DEVERR_CONTEXT and
+ * the sequence's rows are not written; a block id outside the pool sets
+ * PKV_DEVERR_BLOCK_ID and reads as zeros.
+ * Supported: head_size 64 or 128, block_size 16 or 32, G in {1, 2, 4, 8},
+ * num_blocks * num_kv_heads * block_size < 2^31.  f32: PKV_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------- */
+pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   const int32_t* context_lens, const int32_t* query_start_loc,
+                                   float scale, int num_tokens, int num_seqs, int num_heads,
+                                   int num_kv_heads, int head_size, int block_size,
+                                   int num_blocks, int max_blocks_per_seq, int max_query_len,
+                                   pkv_dtype dtype, void* stream);
+
 pkv_status pkv_read_device_errors(void* stream, uint32_t* bits);
 
 /* ---------------------------------------------------------------------------

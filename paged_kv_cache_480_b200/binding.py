@@ -74,6 +74,8 @@ def load_library(path=LIB_PATH):
         lib.paged_attention_decode_fp8kv.restype = I
         lib.reshape_and_cache_fp8kv.argtypes = [P, P, P, P, P, I, I, I, I, I, I64, I64, I, F, F, P]
         lib.reshape_and_cache_fp8kv.restype = I
+        lib.paged_attention_prefill.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P]
+        lib.paged_attention_prefill.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         lib.pkv_read_device_errors.restype = I
         lib.pkv_bm_create.argtypes = [I, I, P, ctypes.POINTER(P)]
@@ -291,6 +293,37 @@ def paged_attention_decode_fp8kv(out, q, k_cache, v_cache, block_tables, context
         int(partition_size), _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(stream, q.device))
     _check(st, "paged_attention_decode_fp8kv")
+    return out
+
+
+def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                            scale, max_query_len=None, stream=None):
+    """Causal prefill / chunked-prefill attention over the paged cache
+    (paged_attention_prefill in pagedkv.h): q, out [T, H, D] packed by
+    sequence (query_start_loc int32 [S + 1]); the last n_s tokens of each
+    sequence's context_lens[s] cached tokens are its queries."""
+    import torch
+    lib = load_library()
+    T, H, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if out.dtype != q.dtype or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise TypeError("q, caches and out must share one dtype")
+    if (block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32
+            or query_start_loc.dtype != torch.int32):
+        raise TypeError("block_tables, context_lens and query_start_loc must be int32")
+    S = context_lens.numel()
+    if query_start_loc.numel() != S + 1 or block_tables.shape[0] != S:
+        raise ValueError("query_start_loc must be [S + 1] and block_tables [S, MB]")
+    if max_query_len is None:
+        raise ValueError("max_query_len is required (a host-known bound of the queries per sequence)")
+    st = lib.paged_attention_prefill(
+        _contig(out, "out"), _contig(q, "q"), _contig(k_cache, "k_cache"), _contig(v_cache, "v_cache"),
+        _contig(block_tables, "block_tables"), _contig(context_lens, "context_lens"),
+        _contig(query_start_loc, "query_start_loc"), float(scale), T, S, H, Hkv, D, bs, NB,
+        block_tables.shape[1], int(max_query_len), _dtype_code(q), _stream(stream, q.device))
+    _check(st, "paged_attention_prefill")
     return out
 
 

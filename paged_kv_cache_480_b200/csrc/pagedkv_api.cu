@@ -6,6 +6,7 @@
 #include "cache_ops.cuh"
 #include "decode_launch.cuh"
 #include "pagedkv.h"
+#include "prefill.cuh"
 
 namespace {
 
@@ -532,6 +533,58 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
         cudaSuccess)
         return PKV_ERR_CUDA;
     return PKV_OK;
+}
+
+pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   const int32_t* context_lens, const int32_t* query_start_loc,
+                                   float scale, int num_tokens, int num_seqs, int num_heads,
+                                   int num_kv_heads, int head_size, int block_size,
+                                   int num_blocks, int max_blocks_per_seq, int max_query_len,
+                                   pkv_dtype dtype, void* stream) {
+    if (num_tokens < 0 || num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_query_len < 0 || max_query_len > num_tokens)
+        return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (head_size != 64 && head_size != 128) return PKV_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
+    if (num_heads % num_kv_heads != 0 || !valid_group(num_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * num_kv_heads * block_size >= (int64_t)0x7fffffff - block_size)
+        return PKV_ERR_UNSUPPORTED;
+    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (max_query_len == 0) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(block_tables) || !aligned4(context_lens) || !aligned4(query_start_loc))
+        return PKV_ERR_INVALID_ARG;
+    int sms = 0;
+    unsigned int* errors = nullptr;
+    pkv_status st = device_info(&sms, &errors);
+    if (st != PKV_OK) return st;
+    pkv::PrefillArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start_loc = query_start_loc;
+    a.errors = errors;
+    a.scale = scale;
+    a.num_tokens = num_tokens;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_size = head_size;
+    a.block_size = block_size;
+    a.num_blocks = num_blocks;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.max_query_len = max_query_len;
+    a.dtype = dtype;
+    return pkv::launch_prefill(a, static_cast<cudaStream_t>(stream));
 }
 
 pkv_status pkv_read_device_errors(void* stream, uint32_t* bits) {

@@ -1,0 +1,143 @@
+// Paged prefill launch: tensor maps for q and the two caches, one kernel
+// instance per (element type, head size, block size, group size).
+#include <atomic>
+#include <cstring>
+
+#include "prefill.cuh"
+#include "prefill_kernel.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (the
+// library links no driver library).
+EncodeTiledFn encoder() {
+    static std::atomic<EncodeTiledFn> cached{nullptr};
+    EncodeTiledFn fn = cached.load(std::memory_order_acquire);
+    if (fn) return fn;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult found = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &found) != cudaSuccess ||
+        found != cudaDriverEntryPointSuccess || ptr == nullptr)
+        return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    cached.store(fn, std::memory_order_release);
+    return fn;
+}
+
+// Tiled map over a row-major tensor, innermost dimension first; boxes of
+// 64 elements (128 bytes) x ..., 128-byte swizzle, zero fill out of bounds.
+bool encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
+            const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+    const cuuint32_t elem_strides[3] = {1, 1, 1};
+    return fn(map, type, (cuuint32_t)rank, const_cast<void*>(base), dims, strides_bytes, box,
+              elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int BS, int G>
+pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
+    using S = PrefillShape<T, D, BS, G>;
+    EncodeTiledFn fn = encoder();
+    if (!fn) return PKV_ERR_CUDA;
+    const CUtensorMapDataType type =
+        std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const cuuint64_t esz = sizeof(T);
+    alignas(64) CUtensorMap tm_q, tm_k, tm_v;
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.num_heads, (cuuint64_t)a.num_tokens};
+        const cuuint64_t strides[2] = {D * esz, (cuuint64_t)a.num_heads * D * esz};
+        const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)S::QT};
+        if (!encode(fn, &tm_q, type, 3, a.q, dims, strides, box)) return PKV_ERR_CUDA;
+    }
+    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
+    if (rows > 0x7fffffff - BS) return PKV_ERR_UNSUPPORTED;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {D * esz};
+        const cuuint32_t box[2] = {64, (cuuint32_t)BS};
+        if (!encode(fn, &tm_k, type, 2, a.k_cache, dims, strides, box)) return PKV_ERR_CUDA;
+        if (!encode(fn, &tm_v, type, 2, a.v_cache, dims, strides, box)) return PKV_ERR_CUDA;
+    }
+    PrefillParams p;
+    std::memset(&p, 0, sizeof p);
+    p.out = a.out;
+    p.block_tables = a.block_tables;
+    p.context_lens = a.context_lens;
+    p.query_start_loc = a.query_start_loc;
+    p.errors = a.errors;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.num_tokens = a.num_tokens;
+    p.num_seqs = a.num_seqs;
+    p.num_heads = a.num_heads;
+    p.num_kv_heads = a.num_kv_heads;
+    p.num_blocks = a.num_blocks;
+    p.max_blocks_per_seq = a.max_blocks_per_seq;
+    p.q_tiles = (a.max_query_len + S::QT - 1) / S::QT;
+    p.cache_rows = (int)rows;
+    const int64_t grid = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
+    if (grid > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+    auto kernel = paged_prefill_kernel<T, D, BS, G>;
+    static std::atomic<bool> configured[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    if (!configured[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) !=
+            cudaSuccess)
+            return PKV_ERR_CUDA;
+        configured[dev].store(true, std::memory_order_release);
+    }
+    if (launch_pdl(kernel, dim3((unsigned)grid), dim3(kPrefillThreads), S::SMEM, stream, p, tm_q, tm_k,
+                   tm_v) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+template <typename T, int D, int BS>
+pkv_status by_group(const PrefillArgs& a, cudaStream_t stream) {
+    switch (a.num_heads / a.num_kv_heads) {
+        case 1: return run<T, D, BS, 1>(a, stream);
+        case 2: return run<T, D, BS, 2>(a, stream);
+        case 4: return run<T, D, BS, 4>(a, stream);
+        case 8: return run<T, D, BS, 8>(a, stream);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+pkv_status by_block(const PrefillArgs& a, cudaStream_t stream) {
+    switch (a.block_size) {
+        case 16: return by_group<T, D, 16>(a, stream);
+        case 32: return by_group<T, D, 32>(a, stream);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+pkv_status by_head(const PrefillArgs& a, cudaStream_t stream) {
+    switch (a.head_size) {
+        case 64: return by_block<T, 64>(a, stream);
+        case 128: return by_block<T, 128>(a, stream);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+pkv_status launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
+    switch (a.dtype) {
+        case PKV_F16: return by_head<__half>(a, stream);
+        case PKV_BF16: return by_head<__nv_bfloat16>(a, stream);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace pkv

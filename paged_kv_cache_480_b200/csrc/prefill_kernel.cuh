@@ -1,0 +1,358 @@
+// Paged prefill / chunked-prefill attention on the sm_100a tensor cores
+// (tcgen05 MMA, accumulators in tensor memory, operands staged by TMA).
+//
+// Sequence s holds L = context_lens[s] tokens in its blocks; the last n of
+// them are this call's queries (rows query_start_loc[s] .. +n of q), query i
+// at position L - n + i attending causally to keys 0 .. L - n + i ("PyTorch-
+// CUDA-v2.9 image enables PagedAttention", workflow list: prefill writes the
+// prompt's KV into pages; usage: chunked prefill).
+//
+// CTA = (sequence, KV head g, tile of M = 128 rows); a row is a (query,
+// head-of-group) pair, row = query * G + head, so every K/V tile serves the
+// G query heads that share it.  Warps 0-3 own rows 32w .. 32w+31 (their
+// tensor-memory lanes) and run the softmax, one row per thread; warp 4
+// issues the TMA loads and the MMAs.  Per key tile of N = 64 keys:
+//   S_b  = Q K^T        tcgen05.mma, A = Q and B = K from 128-byte-swizzled
+//                       shared memory (K-major), D in tensor memory; two S
+//                       buffers let the QK of tile j+1 run during the
+//                       softmax of tile j;
+//   P    = exp2(S * scale*log2e - m_ref) rounded to the element type,
+//          written over S_b in tensor memory;
+//   O   += P V          tcgen05.mma with A = P from tensor memory and B = V
+//                       from shared memory (MN-major).
+// m_ref is raised (and O and l rescaled) only when a row's maximum grows by
+// more than 8 in log2 units, so O stays exact up to the final division by l.
+// Every wait is bounded; the tensor memory is freed on every path.
+#pragma once
+
+#include <math.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "tc05.cuh"
+
+namespace pkv {
+namespace prefill {
+
+constexpr unsigned kAll = 0xffffffffu;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait taken by all 32 lanes; true only if every lane saw the phase,
+// so a failure leaves the whole warp on the same path.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+    const bool got = mbar_wait_bounded(bar, parity, kWaitLimit);
+    return __all_sync(kAll, got);
+}
+
+}  // namespace prefill
+
+struct PrefillParams {
+    void* out;                        // [T][H][D]
+    const int32_t* block_tables;      // [S][MB]
+    const int32_t* context_lens;      // [S]
+    const int32_t* query_start_loc;   // [S + 1]
+    unsigned int* errors;
+    float scale_log2;
+    int num_tokens, num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq;
+    int q_tiles;                      // query tiles per (sequence, KV head)
+    int cache_rows;                   // rows of the [NB * Hkv * bs][D] view of a cache
+};
+
+template <typename T, int D, int BS, int G>
+struct PrefillShape {
+    static constexpr int M = 128;               // rows per CTA
+    static constexpr int QT = M / G;            // queries per CTA
+    static constexpr int N = 64;                // keys per tile
+    static constexpr int DH = D / 64;           // 64-dim halves (one 128-byte swizzle row each)
+    static constexpr int BPT = N / BS;          // cache blocks per key tile
+    static constexpr int STAGES = D == 64 ? 4 : 3;   // K/V tiles in flight (D = 64: two CTAs per SM)
+    static constexpr uint32_t Q_HALF = M * 128;
+    static constexpr uint32_t KV_HALF = N * 128;
+    static constexpr uint32_t Q_BYTES = DH * Q_HALF;
+    static constexpr uint32_t KV_BYTES = DH * KV_HALF;      // K or V of one tile
+    static constexpr uint32_t OFF_KV = Q_BYTES;             // stage st: K at +2*st*KV_BYTES, V after
+    static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * KV_BYTES;
+    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // barriers, TMEM holder, 1 KB alignment slack
+    static constexpr uint32_t TM_S = 0;                     // S buffers at columns 0 and N (fp32)
+    static constexpr uint32_t TM_O = 2 * N;                 // O at columns 2N .. 2N + D
+    static constexpr uint32_t TM_COLS = 256;
+    static_assert(2 * N + D <= 256, "tensor-memory budget");
+    static_assert(N % BS == 0, "key tile holds whole blocks");
+};
+
+constexpr uint32_t kPrefillThreads = 160;
+
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    using S = PrefillShape<T, D, BS, G>;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+    unsigned char* smem = smem_raw + pad;
+    const uint32_t sm = raw_s + pad;                // 1024-byte aligned shared address
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    griddep_wait();
+    using namespace prefill;
+    // ---- which tile: the later query tiles (more keys) are scheduled first ----
+    const int Hkv = p.num_kv_heads;
+    const int pairs = p.num_seqs * Hkv;
+    const int tile = p.q_tiles - 1 - (int)(blockIdx.x / pairs);
+    const int rest = blockIdx.x % pairs;
+    const int g = rest % Hkv;
+    const int s = rest / Hkv;
+    const int q0 = p.query_start_loc[s];
+    const int n = p.query_start_loc[s + 1] - q0;
+    const int L = p.context_lens[s];
+    const int i0 = tile * S::QT;
+    if (n < 0 || n > L || n > p.q_tiles * S::QT || L > p.max_blocks_per_seq * BS || q0 < 0 ||
+        q0 + n > p.num_tokens) {
+        if (threadIdx.x == 0) flag_error(p.errors, PKV_DEVERR_CONTEXT);
+        return;
+    }
+    if (i0 >= n) return;                            // whole CTA, before any barrier or TMEM use
+    const int i_last = min(i0 + S::QT, n) - 1;
+    const int kmax = L - n + i_last + 1;            // keys 0 .. kmax-1 are needed
+    const int nT = (kmax + S::N - 1) / S::N;
+
+    // ---- barriers and tensor memory ----
+    const uint32_t bar = sm + S::OFF_BAR;
+    const uint32_t bar_q = bar;                     // +0
+    auto bar_kv = [&](int st) { return bar + 8 * (1 + st); };         // STAGES
+    auto bar_s = [&](int b) { return bar + 8 * (1 + S::STAGES + b); };  // 2
+    auto bar_p = [&](int b) { return bar + 8 * (3 + S::STAGES + b); };  // 2
+    auto bar_o = [&](int b) { return bar + 8 * (5 + S::STAGES + b); };  // 2
+    const uint32_t bar_fin = bar + 8 * (7 + S::STAGES);
+    uint32_t* tm_holder = reinterpret_cast<uint32_t*>(smem + S::OFF_BAR + 128);
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int st = 0; st < S::STAGES; ++st) mbar_init(bar_kv(st), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_s(b), 1);
+            mbar_init(bar_p(b), 128);
+            mbar_init(bar_o(b), 1);
+        }
+        mbar_init(bar_fin, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc05::tmem_alloc(smem_addr(tm_holder), S::TM_COLS);
+        tc05::tmem_relinquish();
+    }
+    tc05::fence_before_sync();
+    __syncthreads();
+    tc05::fence_after_sync();
+    const uint32_t tm = *tm_holder;
+    bool ok = true;
+
+    const uint32_t q_base = sm;
+    auto k_base = [&](int st) { return sm + S::OFF_KV + (uint32_t)st * 2 * S::KV_BYTES; };
+    auto v_base = [&](int st) { return k_base(st) + S::KV_BYTES; };
+
+    if (warp == 4) {
+        // ===================== control warp: TMA and MMA issue =====================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = tc05::instr_desc(kBf16, 128, S::N, false, false);
+            constexpr uint32_t idesc_pv = tc05::instr_desc(kBf16, 128, D, false, true);
+            const int nblk_seq = (L + BS - 1) / BS;
+            int issued = 0, landed = 0;             // K/V tiles requested / seen complete
+            bool q_landed = false;
+            auto issue_kv = [&](int t) {
+                issued = t + 1;
+                const int st = t % S::STAGES;
+                mbar_arrive_expect_tx(bar_kv(st), 2 * S::KV_BYTES);
+                for (int bi = 0; bi < S::BPT; ++bi) {
+                    const int lb = t * S::BPT + bi;
+                    int row = p.cache_rows;                   // past the end: TMA fills zeros
+                    if (lb < nblk_seq) {
+                        const int phys = p.block_tables[(size_t)s * p.max_blocks_per_seq + lb];
+                        if (phys >= 0 && phys < p.num_blocks) row = (phys * Hkv + g) * BS;
+                        else flag_error(p.errors, PKV_DEVERR_BLOCK_ID);
+                    }
+                    for (int dh = 0; dh < S::DH; ++dh) {
+                        const uint32_t off = dh * S::KV_HALF + bi * BS * 128;
+                        tc05::tma_load_2d(k_base(st) + off, &tm_k, dh * 64, row, bar_kv(st));
+                        tc05::tma_load_2d(v_base(st) + off, &tm_v, dh * 64, row, bar_kv(st));
+                    }
+                }
+            };
+            auto issue_pv = [&](int j) -> bool {
+                const int b = j & 1, st = j % S::STAGES;
+                if (!mbar_wait_bounded(bar_p(b), (j >> 1) & 1, kWaitLimit)) return false;
+                tc05::fence_after_sync();
+                for (int k = 0; k < S::N / 16; ++k) {
+                    const uint64_t vd = tc05::smem_desc(v_base(st) + k * 16 * 128, S::KV_HALF, 1024);
+                    tc05::mma_ts(tm + S::TM_O, tm + S::TM_S + b * S::N + 8 * k, vd, idesc_pv,
+                                 (j > 0 || k > 0) ? 1u : 0u);
+                }
+                tc05::commit(bar_o(b));
+                if (j + S::STAGES < nT) {              // the stage is free once PV(j) is done
+                    if (!mbar_wait_bounded(bar_o(b), (j >> 1) & 1, kWaitLimit)) return false;
+                    issue_kv(j + S::STAGES);
+                }
+                return true;
+            };
+
+            mbar_arrive_expect_tx(bar_q, S::Q_BYTES);
+            for (int dh = 0; dh < S::DH; ++dh)
+                tc05::tma_load_3d(q_base + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0, bar_q);
+            for (int t = 0; t < S::STAGES && t < nT; ++t) issue_kv(t);
+            ok = q_landed = mbar_wait_bounded(bar_q, 0, kWaitLimit);
+            for (int j = 0; ok && j < nT; ++j) {
+                const int b = j & 1, st = j % S::STAGES;
+                if (!mbar_wait_bounded(bar_kv(st), (j / S::STAGES) & 1, kWaitLimit)) { ok = false; break; }
+                landed = j + 1;
+                if (j >= 2 && !mbar_wait_bounded(bar_o(b), ((j - 2) >> 1) & 1, kWaitLimit)) { ok = false; break; }
+                tc05::fence_after_sync();
+                for (int k = 0; k < D / 16; ++k) {
+                    const int dh = k >> 2, kk = k & 3;
+                    const uint64_t ad = tc05::smem_desc(q_base + dh * S::Q_HALF + kk * 32, 16, 1024);
+                    const uint64_t bd = tc05::smem_desc(k_base(st) + dh * S::KV_HALF + kk * 32, 16, 1024);
+                    tc05::mma_ss(tm + S::TM_S + b * S::N, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                }
+                tc05::commit(bar_s(b));
+                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok && !issue_pv(nT - 1)) ok = false;
+            if (!ok) {
+                // a wait gave up: let the copies already requested land before the CTA exits
+                flag_error(p.errors, PKV_DEVERR_WAIT);
+                if (!q_landed) mbar_wait_bounded(bar_q, 0, kWaitLimit);
+                for (int t = landed; t < issued; ++t)
+                    mbar_wait_bounded(bar_kv(t % S::STAGES), (t / S::STAGES) & 1, kWaitLimit);
+            }
+            // every MMA issued above is complete before the tensor memory is freed
+            tc05::commit(bar_fin);
+            mbar_wait_bounded(bar_fin, 0, kWaitLimit);
+        }
+    } else {
+        // ===================== softmax warps: one row per thread =====================
+        const int r = warp * 32 + lane;
+        const int qi = i0 + r / G;                      // query of this row
+        const bool valid = qi < n;
+        const int pos = valid ? L - n + qi : -1;        // keys 0 .. pos are visible
+        const uint32_t trow = tm + ((uint32_t)(warp * 32) << 16);
+        float m_ref = -INFINITY, l = 0.f;
+        for (int j = 0; j < nT; ++j) {
+            const int b = j & 1;
+            if (!warp_wait(bar_s(b), (j >> 1) & 1)) { ok = false; break; }
+            tc05::fence_after_sync();
+            uint32_t sv[64];
+            tc05::tmem_ld32(trow + S::TM_S + b * S::N, *reinterpret_cast<uint32_t(*)[32]>(sv));
+            tc05::tmem_ld32(trow + S::TM_S + b * S::N + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            tc05::tmem_wait_ld();
+            const int key0 = j * S::N;
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float z = (key0 + c <= pos) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+                sv[c] = __float_as_uint(z);
+                mt = fmaxf(mt, z);
+            }
+            const bool raise = mt > m_ref + 8.f;
+            const float new_ref = raise ? mt : m_ref;
+            const float alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
+            l *= alpha;
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float z0 = __uint_as_float(sv[2 * c]), z1 = __uint_as_float(sv[2 * c + 1]);
+                const float p0 = (z0 == -INFINITY) ? 0.f : ex2(z0 - new_ref);
+                const float p1 = (z1 == -INFINITY) ? 0.f : ex2(z1 - new_ref);
+                pk[c] = Elem<T>::pack2(p0, p1);
+                float a, bb;
+                if constexpr (kBf16) {
+                    Elem<__nv_bfloat16>::widen2(pk[c], a, bb);
+                } else {
+                    Elem<__half>::widen2(pk[c], a, bb);
+                }
+                l += a + bb;
+            }
+            // O holds PV of tiles < j: rescale rows whose reference moved (after PV(j-1) is done)
+            if (j >= 1 && __any_sync(kAll, alpha != 1.f)) {
+                if (!warp_wait(bar_o((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+                tc05::fence_after_sync();
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ov[32];
+                    tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
+                    tc05::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
+                }
+                tc05::tmem_wait_st();
+            }
+            // last tile: V rows past the context may hold anything (NaN * 0 = NaN): zero them
+            if (j == nT - 1 && L < (j + 1) * S::N) {
+                const int st = j % S::STAGES;
+                if (!warp_wait(bar_kv(st), (j / S::STAGES) & 1)) { ok = false; break; }
+                const int r0 = max(L - j * S::N, 0);
+                const int chunks = (S::N - r0) * S::DH * 8;     // 16-byte chunks
+                for (int c = r; c < chunks; c += 128) {
+                    const int dh = c / ((S::N - r0) * 8);
+                    const int rem = c - dh * (S::N - r0) * 8;
+                    const int row = r0 + rem / 8, ch = rem % 8;
+                    *reinterpret_cast<uint4*>(smem + (v_base(st) - sm) + dh * S::KV_HALF + row * 128 + ch * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async();
+            }
+            tc05::tmem_st32(trow + S::TM_S + b * S::N, pk);      // P over S (this row only)
+            tc05::tmem_wait_st();
+            tc05::fence_before_sync();
+            mbar_arrive(bar_p(b));
+            m_ref = new_ref;
+        }
+        // ---- epilogue: O / l to the output ----
+        if (ok && warp_wait(bar_o((nT - 1) & 1), ((nT - 1) >> 1) & 1)) {
+            tc05::fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            T* orow = reinterpret_cast<T*>(p.out) +
+                      ((size_t)(q0 + qi) * p.num_heads + (size_t)g * G + (r % G)) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t ov[32];
+                tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
+                tc05::tmem_wait_ld();
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = Elem<T>::pack2(__uint_as_float(ov[8 * v + 2 * e]) * inv,
+                                                  __uint_as_float(ov[8 * v + 2 * e + 1]) * inv);
+                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        } else if (ok) {
+            ok = false;
+        }
+        if (!ok && lane == 0) flag_error(p.errors, PKV_DEVERR_WAIT);
+    }
+    griddep_launch();
+    tc05::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc05::fence_after_sync();
+        tc05::tmem_dealloc(tm, S::TM_COLS);
+    }
+}
+
+}  // namespace pkv

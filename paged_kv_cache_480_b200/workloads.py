@@ -356,3 +356,102 @@ def cow_queries(sc, device="cpu"):
     gen = torch.Generator(device=device)
     gen.manual_seed(sc.seed * 1000 + 17)
     return _randn(gen, (sc.num_seqs, sc.num_heads, sc.head_size), device, 1.0, sc.dtype)
+
+
+# ---------------------------------------------------------------------------
+# Prefill / chunked prefill.
+# ---------------------------------------------------------------------------
+PREFILL_CONFIGS = {
+    # whole prompts of a Llama-2-7B-shaped layer (32 heads, head 128): n = L
+    "prefill_llama7b_bf16": dict(index=5, num_seqs=16, num_heads=32, num_kv_heads=32, head_size=128,
+                                 block_size=16, dtype="bf16"),
+    # the last 512-token chunk of long prompts, 64 query heads over 8 KV heads
+    "chunked_gqa_bf16": dict(index=6, num_seqs=16, num_heads=64, num_kv_heads=8, head_size=128,
+                             block_size=16, dtype="bf16"),
+}
+
+
+def make_prefill_layout(name=None, seed=None, num_seqs=None, max_context=None, context_lens=None,
+                        query_lens=None, dtype=None, num_heads=None, num_kv_heads=None, head_size=None,
+                        block_size=None, chunk=512):
+    """Integer structure of one prefill call.
+
+    prefill_llama7b_bf16: lengths U{512..2048}, every token a query (n = L).
+    chunked_gqa_bf16: contexts U{4096..16384}, the last min(chunk, L)
+    tokens are the queries (earlier chunks already in the cache).
+    Without a name, context_lens / query_lens and the shape arguments give
+    the call directly.  The pool is 1.1x the blocks in use, ids shuffled.
+    ``extra['query_lens']`` holds n per sequence and
+    ``extra['query_start_loc']`` their prefix sums (int32 [S + 1]).
+    """
+    if name is not None:
+        cfg = dict(PREFILL_CONFIGS[name])
+        idx = cfg.pop("index")
+        seed = BASE_SEED + idx if seed is None else seed
+    else:
+        cfg = dict(num_seqs=len(context_lens), num_heads=num_heads, num_kv_heads=num_kv_heads,
+                   head_size=head_size, block_size=block_size, dtype=dtype)
+        seed = BASE_SEED if seed is None else seed
+    for k, v in dict(num_seqs=num_seqs, num_heads=num_heads, num_kv_heads=num_kv_heads,
+                     head_size=head_size, block_size=block_size, dtype=dtype).items():
+        if v is not None:
+            cfg[k] = v
+    rng = np.random.default_rng(seed)
+    S, bs, D = cfg["num_seqs"], cfg["block_size"], cfg["head_size"]
+    if context_lens is not None:
+        lens = np.asarray(context_lens, np.int64)
+        S = len(lens)
+    elif name == "prefill_llama7b_bf16":
+        lens = rng.integers(512, 2049, S)
+    elif name == "chunked_gqa_bf16":
+        lens = rng.integers(4096, 16385, S)
+    else:
+        raise ValueError("context_lens is required without a named workload")
+    if max_context is not None:
+        lens = np.minimum(lens, max_context)
+    lens = lens.astype(np.int32)
+    if query_lens is not None:
+        nq = np.asarray(query_lens, np.int32)
+    elif name == "chunked_gqa_bf16":
+        nq = np.minimum(lens, chunk).astype(np.int32)
+    else:
+        nq = lens.copy()
+    if len(nq) != S or np.any(nq < 0) or np.any(nq > lens):
+        raise ValueError("query_lens must satisfy 0 <= n <= context_len per sequence")
+    used = int(sum(-(-int(L) // bs) for L in lens))
+    nb = max(int(math.ceil(1.1 * used)), used + 1)
+    ids = rng.permutation(nb)[:used]
+    tables = _tables_from_ids(lens, bs, ids)
+    qsl = np.concatenate([[0], np.cumsum(nq.astype(np.int64))]).astype(np.int32)
+    return Layout(name=name or "custom_prefill", dtype=cfg["dtype"], num_seqs=S,
+                  num_heads=cfg["num_heads"], num_kv_heads=cfg["num_kv_heads"], head_size=D,
+                  block_size=bs, num_blocks=nb, scale=1.0 / math.sqrt(D), value_scale=1.0,
+                  context_lens=lens, block_tables=tables, slot_mapping=_slots(lens, tables, bs),
+                  seed=seed, extra=dict(query_lens=nq, query_start_loc=qsl))
+
+
+def make_prefill_tensors(layout, device="cpu"):
+    """q [T,H,D] and k_cache/v_cache [NB,Hkv,bs,D] with every context token
+    (queries' own keys included) already in the pool; other slots NaN."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(layout.seed * 1000 + 19)
+    T = int(layout.extra["query_start_loc"][-1])
+    H, Hkv, D = layout.num_heads, layout.num_kv_heads, layout.head_size
+    NB, bs = layout.num_blocks, layout.block_size
+    vs = layout.value_scale
+    q = _randn(gen, (T, H, D), device, vs, layout.dtype)
+    k_cache = _randn(gen, (NB, Hkv, bs, D), device, vs, layout.dtype)
+    v_cache = _randn(gen, (NB, Hkv, bs, D), device, vs, layout.dtype)
+    invalid = torch.from_numpy(~valid_slot_mask(layout, include_new_token=True)).to(device)
+    k_cache.masked_fill_(invalid[:, None, :, None], float("nan"))
+    v_cache.masked_fill_(invalid[:, None, :, None], float("nan"))
+    return dict(q=q, k_cache=k_cache, v_cache=v_cache)
+
+
+def prefill_pairs(layout):
+    """(query, key) pairs the causal mask keeps: sum over queries of L - n + i + 1."""
+    total = 0
+    for L, n in zip(layout.context_lens.astype(np.int64), layout.extra["query_lens"].astype(np.int64)):
+        total += n * (L - n) + n * (n + 1) // 2
+    return int(total)

@@ -100,3 +100,30 @@ def test_cache_ops_reject_bad_arguments(lib):
     null = (ctypes.c_void_p * 1)(0)
     assert lib.copy_blocks(null, null, 1, P(16), 2, 8, 1024, None) == 1
     assert lib.copy_blocks(arr, arr, 1, P(16), 0, 8, 1024, None) == 0   # nothing to copy
+
+
+def _prefill(lib, **kw):
+    args = dict(out=16, q=16, k=16, v=16, bt=16, cl=16, qsl=16, scale=0.1, t=40, s=2, h=4, hkv=4, d=64,
+                bs=16, nb=8, mb=4, mq=32, dtype=2)
+    args.update(kw)
+    P = ctypes.c_void_p
+    return lib.paged_attention_prefill(
+        P(args["out"]), P(args["q"]), P(args["k"]), P(args["v"]), P(args["bt"]), P(args["cl"]),
+        P(args["qsl"]), args["scale"], args["t"], args["s"], args["h"], args["hkv"], args["d"], args["bs"],
+        args["nb"], args["mb"], args["mq"], args["dtype"], None)
+
+
+def test_prefill_rejects_bad_arguments_before_launch(lib):
+    assert _prefill(lib, out=0) == 1                 # null pointer
+    assert _prefill(lib, qsl=0) == 1
+    assert _prefill(lib, dtype=0) == 2               # f32: no tensor-core kernel
+    assert _prefill(lib, d=96) == 2                  # head size
+    assert _prefill(lib, bs=8) == 2                  # block size
+    assert _prefill(lib, h=12, hkv=1) == 2           # G = 12
+    assert _prefill(lib, q=8) == 1                   # misaligned q
+    assert _prefill(lib, qsl=18) == 1                # misaligned int32 array
+    assert _prefill(lib, mq=41) == 1                 # bound above the token count
+    assert _prefill(lib, mq=0) == 1                  # tokens but no queries bound
+    assert _prefill(lib, scale=float("nan")) == 1
+    assert _prefill(lib, nb=1 << 27, hkv=4) == 2     # pool rows beyond 2^31
+    assert _prefill(lib, t=0, mq=0) == 0             # nothing to do
