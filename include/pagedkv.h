@@ -343,6 +343,7 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
  *                  including this call's queries (written beforehand)
  *   query_start_loc device, int32 [num_seqs + 1], non-decreasing,
  *                  query_start_loc[0] = 0, query_start_loc[num_seqs] = num_tokens
+ *   scale          softmax scale, finite and > 0 (else PKV_ERR_INVALID_ARG)
  *   max_query_len  host-known bound of n over the batch (> 0 unless
  *                  num_tokens == 0); sizes the grid
  *   dtype          f16 or bf16 (q, caches and out the same); the products

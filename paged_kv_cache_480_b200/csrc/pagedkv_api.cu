@@ -1,6 +1,7 @@
 // C-ABI entry points: argument checks on the host, launch planning, and the
 // sticky device-check flag.  Nothing here allocates device memory.
 #include <atomic>
+#include <cmath>
 #include <cstring>
 
 #include "cache_ops.cuh"
@@ -551,7 +552,7 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
     if (num_heads % num_kv_heads != 0 || !valid_group(num_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
     if ((int64_t)num_blocks * num_kv_heads * block_size >= (int64_t)0x7fffffff - block_size)
         return PKV_ERR_UNSUPPORTED;
-    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < INFINITY)) return PKV_ERR_INVALID_ARG;
     if (num_tokens == 0) return PKV_OK;
     if (max_query_len == 0) return PKV_ERR_INVALID_ARG;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)

@@ -11,7 +11,9 @@
 // head-of-group) pair, row = query * G + head, so every K/V tile serves the
 // G query heads that share it.  Warps 0-3 own rows 32w .. 32w+31 (their
 // tensor-memory lanes) and run the softmax, one row per thread; warp 4
-// issues the TMA loads and the MMAs.  Per key tile of N = 64 keys:
+// issues the MMAs; warp 5 streams K/V tiles through a ring of stages with
+// TMA, refilling a stage as soon as the MMA that read it is done.  Per key
+// tile of N = 64 keys:
 //   S_b  = Q K^T        tcgen05.mma, A = Q and B = K from 128-byte-swizzled
 //                       shared memory (K-major), D in tensor memory; two S
 //                       buffers let the QK of tile j+1 run during the
@@ -22,6 +24,7 @@
 //                       from shared memory (MN-major).
 // m_ref is raised (and O and l rescaled) only when a row's maximum grows by
 // more than 8 in log2 units, so O stays exact up to the final division by l.
+// Masks are applied only on tiles that reach past some row's position.
 // Every wait is bounded; the tensor memory is freed on every path.
 #pragma once
 
@@ -62,11 +65,15 @@ struct PrefillParams {
     const int32_t* context_lens;      // [S]
     const int32_t* query_start_loc;   // [S + 1]
     unsigned int* errors;
-    float scale_log2;
+    float scale_log2;                 // softmax scale * log2(e), > 0
     int num_tokens, num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq;
     int q_tiles;                      // query tiles per (sequence, KV head)
     int cache_rows;                   // rows of the [NB * Hkv * bs][D] view of a cache
 };
+
+#ifndef PKV_PREFILL_STAGES_D128
+#define PKV_PREFILL_STAGES_D128 4
+#endif
 
 template <typename T, int D, int BS, int G>
 struct PrefillShape {
@@ -75,28 +82,32 @@ struct PrefillShape {
     static constexpr int N = 64;                // keys per tile
     static constexpr int DH = D / 64;           // 64-dim halves (one 128-byte swizzle row each)
     static constexpr int BPT = N / BS;          // cache blocks per key tile
-    static constexpr int STAGES = D == 64 ? 4 : 3;   // K/V tiles in flight (D = 64: two CTAs per SM)
+    static constexpr int STAGES = D == 64 ? 4 : PKV_PREFILL_STAGES_D128;   // K/V tiles in flight
     static constexpr uint32_t Q_HALF = M * 128;
     static constexpr uint32_t KV_HALF = N * 128;
     static constexpr uint32_t Q_BYTES = DH * Q_HALF;
     static constexpr uint32_t KV_BYTES = DH * KV_HALF;      // K or V of one tile
     static constexpr uint32_t OFF_KV = Q_BYTES;             // stage st: K at +2*st*KV_BYTES, V after
     static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * KV_BYTES;
-    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // barriers, TMEM holder, 1 KB alignment slack
+    static constexpr uint32_t SMEM = OFF_BAR + 512 + 1024;  // barriers, TMEM holder, 1 KB alignment slack
     static constexpr uint32_t TM_S = 0;                     // S buffers at columns 0 and N (fp32)
     static constexpr uint32_t TM_O = 2 * N;                 // O at columns 2N .. 2N + D
     static constexpr uint32_t TM_COLS = 256;
     static_assert(2 * N + D <= 256, "tensor-memory budget");
     static_assert(N % BS == 0, "key tile holds whole blocks");
+    static_assert(8 * (8 + 2 * STAGES) <= 256, "barrier area");
 };
 
-constexpr uint32_t kPrefillThreads = 160;
+// warps 0-3 softmax, warp 4 MMA issue, warp 5 TMA loads
+constexpr uint32_t kPrefillThreads = 192;
 
 template <typename T, int D, int BS, int G>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     using S = PrefillShape<T, D, BS, G>;
+    using namespace prefill;
+    constexpr int ST = S::STAGES;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
@@ -106,7 +117,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     griddep_wait();
-    using namespace prefill;
     // ---- which tile: the later query tiles (more keys) are scheduled first ----
     const int Hkv = p.num_kv_heads;
     const int pairs = p.num_seqs * Hkv;
@@ -130,16 +140,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     // ---- barriers and tensor memory ----
     const uint32_t bar = sm + S::OFF_BAR;
-    const uint32_t bar_q = bar;                     // +0
-    auto bar_kv = [&](int st) { return bar + 8 * (1 + st); };         // STAGES
-    auto bar_s = [&](int b) { return bar + 8 * (1 + S::STAGES + b); };  // 2
-    auto bar_p = [&](int b) { return bar + 8 * (3 + S::STAGES + b); };  // 2
-    auto bar_o = [&](int b) { return bar + 8 * (5 + S::STAGES + b); };  // 2
-    const uint32_t bar_fin = bar + 8 * (7 + S::STAGES);
-    uint32_t* tm_holder = reinterpret_cast<uint32_t*>(smem + S::OFF_BAR + 128);
+    const uint32_t bar_q = bar;
+    auto bar_full = [&](int st) { return bar + 8 * (1 + st); };           // K/V tile landed
+    auto bar_empty = [&](int st) { return bar + 8 * (1 + ST + st); };     // its PV is done
+    auto bar_s = [&](int b) { return bar + 8 * (1 + 2 * ST + b); };       // S_b written
+    auto bar_p = [&](int b) { return bar + 8 * (3 + 2 * ST + b); };       // P_b written (128 threads)
+    auto bar_o = [&](int b) { return bar + 8 * (5 + 2 * ST + b); };       // PV of a b-tile done
+    const uint32_t bar_fin = bar + 8 * (7 + 2 * ST);
+    uint32_t* tm_holder = reinterpret_cast<uint32_t*>(smem + S::OFF_BAR + 256);
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int st = 0; st < S::STAGES; ++st) mbar_init(bar_kv(st), 1);
+        for (int st = 0; st < ST; ++st) {
+            mbar_init(bar_full(st), 1);
+            mbar_init(bar_empty(st), 1);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_s(b), 1);
             mbar_init(bar_p(b), 128);
@@ -156,24 +170,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     __syncthreads();
     tc05::fence_after_sync();
     const uint32_t tm = *tm_holder;
-    bool ok = true;
 
     const uint32_t q_base = sm;
     auto k_base = [&](int st) { return sm + S::OFF_KV + (uint32_t)st * 2 * S::KV_BYTES; };
     auto v_base = [&](int st) { return k_base(st) + S::KV_BYTES; };
 
-    if (warp == 4) {
-        // ===================== control warp: TMA and MMA issue =====================
+    if (warp == 5) {
+        // ===================== TMA producer =====================
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = tc05::instr_desc(kBf16, 128, S::N, false, false);
-            constexpr uint32_t idesc_pv = tc05::instr_desc(kBf16, 128, D, false, true);
             const int nblk_seq = (L + BS - 1) / BS;
-            int issued = 0, landed = 0;             // K/V tiles requested / seen complete
-            bool q_landed = false;
-            auto issue_kv = [&](int t) {
-                issued = t + 1;
-                const int st = t % S::STAGES;
-                mbar_arrive_expect_tx(bar_kv(st), 2 * S::KV_BYTES);
+            mbar_arrive_expect_tx(bar_q, S::Q_BYTES);
+            for (int dh = 0; dh < S::DH; ++dh)
+                tc05::tma_load_3d(q_base + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0, bar_q);
+            int issued = 0;
+            for (int t = 0; t < nT; ++t) {
+                const int st = t % ST;
+                if (t >= ST && !mbar_wait_bounded(bar_empty(st), ((t / ST) - 1) & 1, kWaitLimit)) {
+                    flag_error(p.errors, PKV_DEVERR_WAIT);
+                    break;
+                }
+                mbar_arrive_expect_tx(bar_full(st), 2 * S::KV_BYTES);
                 for (int bi = 0; bi < S::BPT; ++bi) {
                     const int lb = t * S::BPT + bi;
                     int row = p.cache_rows;                   // past the end: TMA fills zeros
@@ -184,68 +200,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                     for (int dh = 0; dh < S::DH; ++dh) {
                         const uint32_t off = dh * S::KV_HALF + bi * BS * 128;
-                        tc05::tma_load_2d(k_base(st) + off, &tm_k, dh * 64, row, bar_kv(st));
-                        tc05::tma_load_2d(v_base(st) + off, &tm_v, dh * 64, row, bar_kv(st));
+                        tc05::tma_load_2d(k_base(st) + off, &tm_k, dh * 64, row, bar_full(st));
+                        tc05::tma_load_2d(v_base(st) + off, &tm_v, dh * 64, row, bar_full(st));
                     }
                 }
-            };
-            auto issue_pv = [&](int j) -> bool {
-                const int b = j & 1, st = j % S::STAGES;
-                if (!mbar_wait_bounded(bar_p(b), (j >> 1) & 1, kWaitLimit)) return false;
-                tc05::fence_after_sync();
-                for (int k = 0; k < S::N / 16; ++k) {
-                    const uint64_t vd = tc05::smem_desc(v_base(st) + k * 16 * 128, S::KV_HALF, 1024);
-                    tc05::mma_ts(tm + S::TM_O, tm + S::TM_S + b * S::N + 8 * k, vd, idesc_pv,
-                                 (j > 0 || k > 0) ? 1u : 0u);
-                }
-                tc05::commit(bar_o(b));
-                if (j + S::STAGES < nT) {              // the stage is free once PV(j) is done
-                    if (!mbar_wait_bounded(bar_o(b), (j >> 1) & 1, kWaitLimit)) return false;
-                    issue_kv(j + S::STAGES);
-                }
-                return true;
-            };
-
-            mbar_arrive_expect_tx(bar_q, S::Q_BYTES);
-            for (int dh = 0; dh < S::DH; ++dh)
-                tc05::tma_load_3d(q_base + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0, bar_q);
-            for (int t = 0; t < S::STAGES && t < nT; ++t) issue_kv(t);
-            ok = q_landed = mbar_wait_bounded(bar_q, 0, kWaitLimit);
-            for (int j = 0; ok && j < nT; ++j) {
-                const int b = j & 1, st = j % S::STAGES;
-                if (!mbar_wait_bounded(bar_kv(st), (j / S::STAGES) & 1, kWaitLimit)) { ok = false; break; }
-                landed = j + 1;
-                if (j >= 2 && !mbar_wait_bounded(bar_o(b), ((j - 2) >> 1) & 1, kWaitLimit)) { ok = false; break; }
-                tc05::fence_after_sync();
-                for (int k = 0; k < D / 16; ++k) {
-                    const int dh = k >> 2, kk = k & 3;
-                    const uint64_t ad = tc05::smem_desc(q_base + dh * S::Q_HALF + kk * 32, 16, 1024);
-                    const uint64_t bd = tc05::smem_desc(k_base(st) + dh * S::KV_HALF + kk * 32, 16, 1024);
-                    tc05::mma_ss(tm + S::TM_S + b * S::N, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
-                }
-                tc05::commit(bar_s(b));
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+                issued = t + 1;
             }
-            if (ok && !issue_pv(nT - 1)) ok = false;
-            if (!ok) {
-                // a wait gave up: let the copies already requested land before the CTA exits
-                flag_error(p.errors, PKV_DEVERR_WAIT);
-                if (!q_landed) mbar_wait_bounded(bar_q, 0, kWaitLimit);
-                for (int t = landed; t < issued; ++t)
-                    mbar_wait_bounded(bar_kv(t % S::STAGES), (t / S::STAGES) & 1, kWaitLimit);
+            // every copy requested above lands before this thread leaves (the last
+            // copy into each stage; earlier ones were consumed before their stage
+            // was refilled)
+            mbar_wait_bounded(bar_q, 0, kWaitLimit);
+            for (int t = max(0, issued - ST); t < issued; ++t)
+                mbar_wait_bounded(bar_full(t % ST), (t / ST) & 1, kWaitLimit);
+        }
+    } else if (warp == 4) {
+        // ===================== MMA issue =====================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = tc05::instr_desc(kBf16, 128, S::N, false, false);
+            constexpr uint32_t idesc_pv = tc05::instr_desc(kBf16, 128, D, false, true);
+            bool ok = mbar_wait_bounded(bar_q, 0, kWaitLimit);
+            for (int j = 0; ok && j <= nT; ++j) {
+                if (j < nT) {                                 // S_b = Q K_j^T
+                    const int b = j & 1, st = j % ST;
+                    if (!mbar_wait_bounded(bar_full(st), (j / ST) & 1, kWaitLimit)) { ok = false; break; }
+                    if (j >= 2 && !mbar_wait_bounded(bar_o(b), ((j - 2) >> 1) & 1, kWaitLimit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc05::fence_after_sync();
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const int dh = k >> 2, kk = k & 3;
+                        const uint64_t ad = tc05::smem_desc(q_base + dh * S::Q_HALF + kk * 32, 16, 1024);
+                        const uint64_t bd = tc05::smem_desc(k_base(st) + dh * S::KV_HALF + kk * 32, 16, 1024);
+                        tc05::mma_ss(tm + S::TM_S + b * S::N, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                    }
+                    tc05::commit(bar_s(b));
+                }
+                if (j >= 1) {                                 // O += P_{j-1} V_{j-1}
+                    const int jj = j - 1, b = jj & 1, st = jj % ST;
+                    if (!mbar_wait_bounded(bar_p(b), (jj >> 1) & 1, kWaitLimit)) { ok = false; break; }
+                    tc05::fence_after_sync();
+#pragma unroll
+                    for (int k = 0; k < S::N / 16; ++k) {
+                        const uint64_t vd = tc05::smem_desc(v_base(st) + k * 16 * 128, S::KV_HALF, 1024);
+                        tc05::mma_ts(tm + S::TM_O, tm + S::TM_S + b * S::N + 8 * k, vd, idesc_pv,
+                                     (jj > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc05::commit(bar_o(b));
+                    tc05::commit(bar_empty(st));
+                }
             }
+            if (!ok) flag_error(p.errors, PKV_DEVERR_WAIT);
             // every MMA issued above is complete before the tensor memory is freed
             tc05::commit(bar_fin);
             mbar_wait_bounded(bar_fin, 0, kWaitLimit);
         }
     } else {
         // ===================== softmax warps: one row per thread =====================
+        bool ok = true;
         const int r = warp * 32 + lane;
         const int qi = i0 + r / G;                      // query of this row
         const bool valid = qi < n;
         const int pos = valid ? L - n + qi : -1;        // keys 0 .. pos are visible
         const uint32_t trow = tm + ((uint32_t)(warp * 32) << 16);
-        float m_ref = -INFINITY, l = 0.f;
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;               // reference max (log2 units), sum of weights
         for (int j = 0; j < nT; ++j) {
             const int b = j & 1;
             if (!warp_wait(bar_s(b), (j >> 1) & 1)) { ok = false; break; }
@@ -255,31 +275,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tc05::tmem_ld32(trow + S::TM_S + b * S::N + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
             tc05::tmem_wait_ld();
             const int key0 = j * S::N;
-            float mt = -INFINITY;
+            if (__any_sync(kAll, key0 + S::N - 1 > pos)) {      // a diagonal (or past-the-end) tile
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float z = (key0 + c <= pos) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-                sv[c] = __float_as_uint(z);
-                mt = fmaxf(mt, z);
+                for (int c = 0; c < 64; ++c)
+                    if (key0 + c > pos) sv[c] = __float_as_uint(-INFINITY);
             }
+            float mx = __uint_as_float(sv[0]);
+#pragma unroll
+            for (int c = 1; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+            const float mt = mx * sl2;                  // the scale is positive
             const bool raise = mt > m_ref + 8.f;
             const float new_ref = raise ? mt : m_ref;
             const float alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
+            const float neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
             l *= alpha;
             uint32_t pk[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const float z0 = __uint_as_float(sv[2 * c]), z1 = __uint_as_float(sv[2 * c + 1]);
-                const float p0 = (z0 == -INFINITY) ? 0.f : ex2(z0 - new_ref);
-                const float p1 = (z1 == -INFINITY) ? 0.f : ex2(z1 - new_ref);
+                const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl2, neg_ref));
+                const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, neg_ref));
+                l += p0 + p1;
                 pk[c] = Elem<T>::pack2(p0, p1);
-                float a, bb;
-                if constexpr (kBf16) {
-                    Elem<__nv_bfloat16>::widen2(pk[c], a, bb);
-                } else {
-                    Elem<__half>::widen2(pk[c], a, bb);
-                }
-                l += a + bb;
             }
             // O holds PV of tiles < j: rescale rows whose reference moved (after PV(j-1) is done)
             if (j >= 1 && __any_sync(kAll, alpha != 1.f)) {
@@ -298,8 +314,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             // last tile: V rows past the context may hold anything (NaN * 0 = NaN): zero them
             if (j == nT - 1 && L < (j + 1) * S::N) {
-                const int st = j % S::STAGES;
-                if (!warp_wait(bar_kv(st), (j / S::STAGES) & 1)) { ok = false; break; }
+                const int st = j % ST;
+                if (!warp_wait(bar_full(st), (j / ST) & 1)) { ok = false; break; }
                 const int r0 = max(L - j * S::N, 0);
                 const int chunks = (S::N - r0) * S::DH * 8;     // 16-byte chunks
                 for (int c = r; c < chunks; c += 128) {
@@ -341,7 +357,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                 }
             }
-        } else if (ok) {
+        } else {
             ok = false;
         }
         if (!ok && lane == 0) flag_error(p.errors, PKV_DEVERR_WAIT);

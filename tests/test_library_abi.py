@@ -125,5 +125,7 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _prefill(lib, mq=41) == 1                 # bound above the token count
     assert _prefill(lib, mq=0) == 1                  # tokens but no queries bound
     assert _prefill(lib, scale=float("nan")) == 1
+    assert _prefill(lib, scale=-0.1) == 1
+    assert _prefill(lib, scale=0.0) == 1
     assert _prefill(lib, nb=1 << 27, hkv=4) == 2     # pool rows beyond 2^31
     assert _prefill(lib, t=0, mq=0) == 0             # nothing to do
