@@ -81,7 +81,7 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     p.num_kv_heads = a.num_kv_heads;
     p.num_blocks = a.num_blocks;
     p.max_blocks_per_seq = a.max_blocks_per_seq;
-    p.q_tiles = (a.max_query_len + S::QT - 1) / S::QT;
+    p.q_tiles = (a.max_query_len + S::CQ - 1) / S::CQ;
     p.cache_rows = (int)rows;
     const int64_t grid = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
     if (grid > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
