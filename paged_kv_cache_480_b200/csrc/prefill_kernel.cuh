@@ -256,6 +256,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = tc05::instr_desc(kBf16, 128, N, false, false);
             constexpr uint32_t idesc_pv = tc05::instr_desc(kBf16, 128, D, false, true);
+            // operand descriptors of query tile 0 and stage 0; the start-address
+            // field (bits 0-13, address / 16) is advanced by plain addition
+            const uint64_t dq = tc05::smem_desc(q_base(0), 16, 1024);
+            const uint64_t dk = tc05::smem_desc(k_base(0), 16, 1024);
+            const uint64_t dv = tc05::smem_desc(v_base(0), S::KV_HALF, 1024);
             bool ok = mbar_wait_bounded(bar_q, 0, kWaitLimit);
             for (int j = 0; ok && j <= nT; ++j) {
                 if (j < nT) {                                 // S_x = Q_x K_j^T
@@ -269,12 +274,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                         tc05::fence_after_sync();
                         const uint32_t d = tm + x * S::TM_TILE + S::TM_S + b * N;
+                        const uint64_t ad = dq + (uint64_t)((x * S::Q_BYTES) >> 4);
+                        const uint64_t bd = dk + (uint64_t)((st * 2 * S::KV_BYTES) >> 4);
+                        // k-th 16-wide slice: +32 bytes inside a swizzle row, next half after 4
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
-                            const int dh = k >> 2, kk = k & 3;
-                            const uint64_t ad = tc05::smem_desc(q_base(x) + dh * S::Q_HALF + kk * 32, 16, 1024);
-                            const uint64_t bd = tc05::smem_desc(k_base(st) + dh * S::KV_HALF + kk * 32, 16, 1024);
-                            tc05::mma_ss(d, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                            const uint32_t qoff = ((k >> 2) * S::Q_HALF + (k & 3) * 32) >> 4;
+                            const uint32_t koff = ((k >> 2) * S::KV_HALF + (k & 3) * 32) >> 4;
+                            tc05::mma_ss(d, ad + qoff, bd + koff, idesc_qk, k > 0 ? 1u : 0u);
                         }
                         tc05::commit(bar_s(x, b));
                     }
@@ -290,12 +297,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                         tc05::fence_after_sync();
                         const uint32_t base = tm + x * S::TM_TILE;
+                        const uint64_t vd = dv + (uint64_t)((st * 2 * S::KV_BYTES) >> 4);
+                        // k-th 16 keys: 16 rows of 128 bytes further
 #pragma unroll
-                        for (int k = 0; k < N / 16; ++k) {
-                            const uint64_t vd = tc05::smem_desc(v_base(st) + k * 16 * 128, S::KV_HALF, 1024);
-                            tc05::mma_ts(base + S::TM_O, base + S::TM_S + b * N + 8 * k, vd, idesc_pv,
-                                         (jj > 0 || k > 0) ? 1u : 0u);
-                        }
+                        for (int k = 0; k < N / 16; ++k)
+                            tc05::mma_ts(base + S::TM_O, base + S::TM_S + b * N + 8 * k, vd + (uint64_t)(k * 128),
+                                         idesc_pv, (jj > 0 || k > 0) ? 1u : 0u);
                         tc05::commit(bar_o(x, b));
                     }
                     if (ok) tc05::commit(bar_empty(st));
