@@ -54,6 +54,36 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) ----
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Bounded wait taken by all 32 lanes; true only if every lane saw the phase,
 // so a failure leaves the whole warp on the same path.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
@@ -78,6 +108,10 @@ struct PrefillParams {
 #ifndef PKV_PREFILL_STAGES
 #define PKV_PREFILL_STAGES 4
 #endif
+#ifndef PKV_PREFILL_ORDER
+#define PKV_PREFILL_ORDER 0
+#endif
+
 
 template <typename T, int D, int BS, int G>
 struct PrefillShape {
@@ -129,8 +163,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- which queries: the later ones (more keys) are scheduled first ----
     const int Hkv = p.num_kv_heads;
     const int pairs = p.num_seqs * Hkv;
+#if PKV_PREFILL_ORDER == 0
     const int tile = p.q_tiles - 1 - (int)(blockIdx.x / pairs);
     const int rest = blockIdx.x % pairs;
+#else
+    // the query tiles of one (sequence, KV head) run side by side and share
+    // its K/V through L2
+    const int tile = p.q_tiles - 1 - (int)(blockIdx.x % p.q_tiles);
+    const int rest = blockIdx.x / p.q_tiles;
+#endif
     const int g = rest % Hkv;
     const int s = rest / Hkv;
     const int q0 = p.query_start_loc[s];
@@ -341,9 +382,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     for (int c = 0; c < 64; ++c)
                         if (key0 + c > pos) sv[c] = __float_as_uint(-INFINITY);
                 }
-                float mx = __uint_as_float(sv[0]);
+                float m4[4];
 #pragma unroll
-                for (int c = 1; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+                for (int a = 0; a < 4; ++a) m4[a] = __uint_as_float(sv[a]);
+#pragma unroll
+                for (int c = 4; c < 64; c += 8)
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        m4[a] = max3(m4[a], __uint_as_float(sv[c + a]), __uint_as_float(sv[c + 4 + a]));
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float mt = mx * sl2;                  // the scale is positive
                 const bool raise = mt > m_ref + 8.f;
                 const float new_ref = raise ? mt : m_ref;
@@ -351,12 +398,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const float neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
                 l *= alpha;
                 uint32_t pk[32];
+                const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
+                uint64_t lsum[4] = {0, 0, 0, 0};         // four packed partial sums (+0.0 bits)
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl2, neg_ref));
-                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, neg_ref));
-                    l += p0 + p1;
+                    const uint64_t z = f2fma(f2pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])),
+                                             sl2x2, refx2);
+                    float z0, z1;
+                    f2unpack(z, z0, z1);
+                    const float p0 = ex2(z0), p1 = ex2(z1);
+                    lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
                     pk[c] = Elem<T>::pack2(p0, p1);
+                }
+                {
+                    float a0, a1, b0, b1, c0, c1, d0, d1;
+                    f2unpack(lsum[0], a0, a1);
+                    f2unpack(lsum[1], b0, b1);
+                    f2unpack(lsum[2], c0, c1);
+                    f2unpack(lsum[3], d0, d1);
+                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
                 }
                 // O holds PV of tiles < j: rescale rows whose reference moved (after PV(j-1) is done)
                 if (j >= 1 && __any_sync(kAll, alpha != 1.f)) {
