@@ -14,22 +14,27 @@
 //   warps 0-3 and 4-7  softmax of query tile 0 and 1, one row per thread
 //                      (warp w reaches tensor-memory lanes 32(w%4) .. +31);
 //   warp 8             issues the MMAs (one thread);
-//   warp 9             streams K/V tiles through a ring of stages with TMA,
-//                      refilling a stage once both tiles' PV products that
-//                      read it are done.
-// Per key tile j of N = 64 keys and query tile x:
-//   S_x,b = Q_x K_j^T   tcgen05.mma, A = Q and B = K from 128-byte-swizzled
-//                       shared memory (K-major), fp32 in tensor memory; two
-//                       S buffers per query tile (b = j mod 2);
-//   P     = exp2(S * scale*log2e - m_ref) rounded to the element type,
-//           written over S_x,b in tensor memory;
-//   O_x  += P V_j       tcgen05.mma with A = P from tensor memory and B = V
-//                       from shared memory (MN-major).
-// While one softmax warpgroup works, the tensor core runs the other tile's
-// products.  m_ref is raised (and O and l rescaled) only when a row's maximum
-// grows by more than 8 in log2 units, so O stays exact up to the final
-// division by l.  Masks are applied only on tiles that reach past some row's
-// position.  Every wait is bounded; the tensor memory is freed on every path.
+//   warps 9 and 10     stream K and V tiles through two rings of stages
+//                      with TMA, each refilling a stage once the products
+//                      that read it are done.
+// Per key tile i of N = 128 keys and query tile x, in tensor memory
+// columns [256x, 256x + 256): S_x (128 fp32 columns), P_x over the first 64
+// of them (16-bit pairs), O_x (D fp32 columns) after S_x:
+//   S_x  = Q_x K_i^T    tcgen05.mma, A = Q and B = K from 128-byte-swizzled
+//                       shared memory (K-major);
+//   P_x  = exp2(S_x * scale*log2e - m_ref) rounded to the element type;
+//   O_x += P_x V_i      tcgen05.mma, A = P from tensor memory, B = V from
+//                       shared memory (MN-major).
+// The MMA thread issues QK_0(i), PV_1(i-1), QK_1(i), PV_0(i): while one
+// softmax warpgroup works on its tile the tensor core runs the other tile's
+// two products.  QK_x(i+1) is issued right behind PV_x(i), whose A operand
+// P_x it overwrites: tcgen05.mma operations of one thread execute in issue
+// order, and a commit covers every earlier operation of its thread, so the
+// softmax that sees S_x(i+1) may also rescale O_x.  m_ref is raised (and O
+// and l rescaled) only when a row's maximum grows by more than 8 in log2
+// units, so O stays exact up to the final division by l.  Masks are applied
+// only on tiles that reach past some row's position.  Every wait is
+// bounded; the tensor memory is freed on every path.
 #pragma once
 
 #include <math.h>
@@ -105,43 +110,43 @@ struct PrefillParams {
     int cache_rows;                   // rows of the [NB * Hkv * bs][D] view of a cache
 };
 
-#ifndef PKV_PREFILL_STAGES
-#define PKV_PREFILL_STAGES 4
-#endif
-#ifndef PKV_PREFILL_ORDER
-#define PKV_PREFILL_ORDER 0
+#ifndef PKV_PREFILL_KST128
+#define PKV_PREFILL_KST128 3
 #endif
 
+#ifndef PKV_PREFILL_VST128
+#define PKV_PREFILL_VST128 2
+#endif
 
 template <typename T, int D, int BS, int G>
 struct PrefillShape {
     static constexpr int M = 128;               // rows per query tile
     static constexpr int QT = M / G;            // queries per query tile
     static constexpr int CQ = 2 * QT;           // queries per CTA
-    static constexpr int N = 64;                // keys per tile
+    static constexpr int N = 128;               // keys per tile
     static constexpr int DH = D / 64;           // 64-dim halves (one 128-byte swizzle row each)
     static constexpr int BPT = N / BS;          // cache blocks per key tile
-    // K/V tiles in flight; with head size 64 the extra stages also keep a
-    // second CTA (and its 512 tensor-memory columns) off the SM
-    static constexpr int STAGES = D == 64 ? 6 : PKV_PREFILL_STAGES;
+    static constexpr int KST = D == 64 ? 4 : PKV_PREFILL_KST128;   // K stages
+    static constexpr int VST = D == 64 ? 4 : PKV_PREFILL_VST128;   // V stages
     static constexpr uint32_t Q_HALF = M * 128;
     static constexpr uint32_t KV_HALF = N * 128;
     static constexpr uint32_t Q_BYTES = DH * Q_HALF;        // one query tile
     static constexpr uint32_t KV_BYTES = DH * KV_HALF;      // K or V of one key tile
-    static constexpr uint32_t OFF_KV = 2 * Q_BYTES;         // stage st: K at +2*st*KV_BYTES, V after
-    static constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * KV_BYTES;
+    static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
     static constexpr uint32_t SMEM = OFF_BAR + 512 + 1024;  // barriers, TMEM holder, 1 KB alignment slack
     static constexpr uint32_t TM_TILE = 256;                // columns per query tile
-    static constexpr uint32_t TM_S = 0;                     // S buffers at columns 0 and N (fp32)
-    static constexpr uint32_t TM_O = 2 * N;                 // O at columns 2N .. 2N + D
+    static constexpr uint32_t TM_S = 0;                     // S (N fp32 columns); P over its first N/2
+    static constexpr uint32_t TM_O = N;                     // O at columns N .. N + D
     static constexpr uint32_t TM_COLS = 512;
-    static_assert(2 * N + D <= (int)TM_TILE, "tensor-memory budget");
+    static_assert(N + D <= (int)TM_TILE, "tensor-memory budget");
     static_assert(N % BS == 0, "key tile holds whole blocks");
-    static_assert(8 * (15 + 2 * STAGES) <= 256, "barrier area");
+    static_assert(8 * (9 + 2 * (KST + VST)) <= 256, "barrier area");
     static_assert(SMEM > 232448 / 2 && SMEM <= 232448, "one CTA per SM");
 };
 
-constexpr uint32_t kPrefillThreads = 320;
+constexpr uint32_t kPrefillThreads = 352;
 
 template <typename T, int D, int BS, int G>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -149,7 +154,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     using S = PrefillShape<T, D, BS, G>;
     using namespace prefill;
-    constexpr int ST = S::STAGES;
+    constexpr int KST = S::KST, VST = S::VST;
     constexpr int N = S::N;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     extern __shared__ unsigned char smem_raw[];
@@ -163,15 +168,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- which queries: the later ones (more keys) are scheduled first ----
     const int Hkv = p.num_kv_heads;
     const int pairs = p.num_seqs * Hkv;
-#if PKV_PREFILL_ORDER == 0
     const int tile = p.q_tiles - 1 - (int)(blockIdx.x / pairs);
     const int rest = blockIdx.x % pairs;
-#else
-    // the query tiles of one (sequence, KV head) run side by side and share
-    // its K/V through L2
-    const int tile = p.q_tiles - 1 - (int)(blockIdx.x % p.q_tiles);
-    const int rest = blockIdx.x / p.q_tiles;
-#endif
     const int g = rest % Hkv;
     const int s = rest / Hkv;
     const int q0 = p.query_start_loc[s];
@@ -188,7 +186,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int nT0 = (L - n + min(i0 + S::QT, n) + N - 1) / N;
     const int nT1 = i0 + S::QT < n ? (L - n + min(i0 + S::CQ, n) + N - 1) / N : 0;
     auto nTx = [&](int x) { return x ? nT1 : nT0; };
-    const int ntiles = nT1 > 0 ? 2 : 1;
+    const bool two = nT1 > 0;
     const int nT = max(nT0, nT1);
     // the last key tile's V rows from the context end to the end of its last
     // block hold whatever the pool holds there; they are zeroed before use
@@ -200,26 +198,32 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- barriers and tensor memory ----
     const uint32_t bar = sm + S::OFF_BAR;
     const uint32_t bar_q = bar;
-    auto bar_full = [&](int st) { return bar + 8 * (1 + st); };                    // K/V tile landed
-    auto bar_empty = [&](int st) { return bar + 8 * (1 + ST + st); };              // its PVs are done
-    auto bar_s = [&](int x, int b) { return bar + 8 * (1 + 2 * ST + 6 * x + b); };   // S written
-    auto bar_p = [&](int x, int b) { return bar + 8 * (3 + 2 * ST + 6 * x + b); };   // P written (128)
-    auto bar_o = [&](int x, int b) { return bar + 8 * (5 + 2 * ST + 6 * x + b); };   // PV done
-    const uint32_t bar_vz = bar + 8 * (13 + 2 * ST);
-    const uint32_t bar_fin = bar + 8 * (14 + 2 * ST);
+    auto bar_kfull = [&](int st) { return bar + 8 * (1 + st); };
+    auto bar_kempty = [&](int st) { return bar + 8 * (1 + KST + st); };
+    auto bar_vfull = [&](int st) { return bar + 8 * (1 + 2 * KST + st); };
+    auto bar_vempty = [&](int st) { return bar + 8 * (1 + 2 * KST + VST + st); };
+    constexpr int B0 = 1 + 2 * KST + 2 * VST;
+    auto bar_s = [&](int x) { return bar + 8 * (B0 + x); };        // QK_x done (and all before it)
+    auto bar_p = [&](int x) { return bar + 8 * (B0 + 2 + x); };    // P_x written (128 arrivals)
+    auto bar_o = [&](int x) { return bar + 8 * (B0 + 4 + x); };    // last PV_x done
+    const uint32_t bar_vz = bar + 8 * (B0 + 6);
+    const uint32_t bar_fin = bar + 8 * (B0 + 7);
     uint32_t* tm_holder = reinterpret_cast<uint32_t*>(smem + S::OFF_BAR + 256);
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int st = 0; st < ST; ++st) {
-            mbar_init(bar_full(st), 1);
-            mbar_init(bar_empty(st), 1);
+        for (int st = 0; st < KST; ++st) {
+            mbar_init(bar_kfull(st), 1);
+            mbar_init(bar_kempty(st), 1);
         }
-        for (int x = 0; x < 2; ++x)
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(bar_s(x, b), 1);
-                mbar_init(bar_p(x, b), 128);
-                mbar_init(bar_o(x, b), 1);
-            }
+        for (int st = 0; st < VST; ++st) {
+            mbar_init(bar_vfull(st), 1);
+            mbar_init(bar_vempty(st), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar_s(x), 1);
+            mbar_init(bar_p(x), 128);
+            mbar_init(bar_o(x), 1);
+        }
         mbar_init(bar_vz, 1);
         mbar_init(bar_fin, 1);
         fence_mbar_init();
@@ -234,52 +238,57 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tm = *tm_holder;
 
     auto q_base = [&](int x) { return sm + (uint32_t)x * S::Q_BYTES; };
-    auto k_base = [&](int st) { return sm + S::OFF_KV + (uint32_t)st * 2 * S::KV_BYTES; };
-    auto v_base = [&](int st) { return k_base(st) + S::KV_BYTES; };
+    auto k_base = [&](int st) { return sm + S::OFF_K + (uint32_t)st * S::KV_BYTES; };
+    auto v_base = [&](int st) { return sm + S::OFF_V + (uint32_t)st * S::KV_BYTES; };
 
-    if (warp == 9) {
-        // ===================== TMA producer =====================
+    if (warp >= 9) {
+        // ===================== TMA producers: warp 9 Q and K, warp 10 V =====================
+        const bool is_v = warp == 10;
         int issued = 0;
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar_q, ntiles * S::Q_BYTES);
-            for (int x = 0; x < ntiles; ++x)
-                for (int dh = 0; dh < S::DH; ++dh)
-                    tc05::tma_load_3d(q_base(x) + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0 + x * S::QT,
-                                      bar_q);
+            if (!is_v) {
+                mbar_arrive_expect_tx(bar_q, (two ? 2 : 1) * S::Q_BYTES);
+                for (int x = 0; x < (two ? 2 : 1); ++x)
+                    for (int dh = 0; dh < S::DH; ++dh)
+                        tc05::tma_load_3d(q_base(x) + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0 + x * S::QT,
+                                          bar_q);
+            }
+            const int nst = is_v ? VST : KST;
+            const CUtensorMap* map = is_v ? &tm_v : &tm_k;
             for (int t = 0; t < nT; ++t) {
-                const int st = t % ST;
-                if (t >= ST && !mbar_wait_bounded(bar_empty(st), ((t / ST) - 1) & 1, kWaitLimit)) {
+                const int st = t % nst;
+                const uint32_t empty = is_v ? bar_vempty(st) : bar_kempty(st);
+                const uint32_t full = is_v ? bar_vfull(st) : bar_kfull(st);
+                const uint32_t dst = is_v ? v_base(st) : k_base(st);
+                if (t >= nst && !mbar_wait_bounded(empty, ((t / nst) - 1) & 1, kWaitLimit)) {
                     flag_error(p.errors, PKV_DEVERR_WAIT);
                     break;
                 }
-                mbar_arrive_expect_tx(bar_full(st), 2 * S::KV_BYTES);
+                mbar_arrive_expect_tx(full, S::KV_BYTES);
                 for (int bi = 0; bi < S::BPT; ++bi) {
                     const int lb = t * S::BPT + bi;
                     int row = p.cache_rows;                   // past the end: TMA fills zeros
                     if (lb < nblk_seq) {
                         const int phys = p.block_tables[(size_t)s * p.max_blocks_per_seq + lb];
                         if (phys >= 0 && phys < p.num_blocks) row = (phys * Hkv + g) * BS;
-                        else flag_error(p.errors, PKV_DEVERR_BLOCK_ID);
+                        else if (!is_v) flag_error(p.errors, PKV_DEVERR_BLOCK_ID);
                     }
-                    for (int dh = 0; dh < S::DH; ++dh) {
-                        const uint32_t off = dh * S::KV_HALF + bi * BS * 128;
-                        tc05::tma_load_2d(k_base(st) + off, &tm_k, dh * 64, row, bar_full(st));
-                        tc05::tma_load_2d(v_base(st) + off, &tm_v, dh * 64, row, bar_full(st));
-                    }
+                    for (int dh = 0; dh < S::DH; ++dh)
+                        tc05::tma_load_2d(dst + dh * S::KV_HALF + bi * BS * 128, map, dh * 64, row, full);
                 }
                 issued = t + 1;
             }
             // every copy requested above lands before this warp leaves (the last
             // copy into each stage; earlier ones were consumed before their stage
             // was refilled)
-            mbar_wait_bounded(bar_q, 0, kWaitLimit);
-            for (int t = max(0, issued - ST); t < issued; ++t)
-                mbar_wait_bounded(bar_full(t % ST), (t / ST) & 1, kWaitLimit);
+            if (!is_v) mbar_wait_bounded(bar_q, 0, kWaitLimit);
+            for (int t = max(0, issued - nst); t < issued; ++t)
+                mbar_wait_bounded(is_v ? bar_vfull(t % nst) : bar_kfull(t % nst), (t / nst) & 1, kWaitLimit);
         }
         issued = __shfl_sync(kAll, issued, 0);
-        if (need_vz && issued == nT) {
-            const int st = (nT - 1) % ST;
-            if (warp_wait(bar_full(st), ((nT - 1) / ST) & 1)) {
+        if (is_v && need_vz && issued == nT) {
+            const int st = (nT - 1) % VST;
+            if (warp_wait(bar_vfull(st), ((nT - 1) / VST) & 1)) {
                 const int rows = vz_r1 - vz_r0;
                 for (int c = lane; c < rows * S::DH * 8; c += 32) {   // 16-byte chunks
                     const int dh = c / (rows * 8);
@@ -303,51 +312,57 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint64_t dk = tc05::smem_desc(k_base(0), 16, 1024);
             const uint64_t dv = tc05::smem_desc(v_base(0), S::KV_HALF, 1024);
             bool ok = mbar_wait_bounded(bar_q, 0, kWaitLimit);
-            for (int j = 0; ok && j <= nT; ++j) {
-                if (j < nT) {                                 // S_x = Q_x K_j^T
-                    const int b = j & 1, st = j % ST;
-                    ok = mbar_wait_bounded(bar_full(st), (j / ST) & 1, kWaitLimit);
-                    for (int x = 0; ok && x < 2; ++x) {
-                        if (j >= nTx(x)) continue;
-                        if (j >= 2 && !mbar_wait_bounded(bar_o(x, b), ((j - 2) >> 1) & 1, kWaitLimit)) {
-                            ok = false;
-                            break;
-                        }
-                        tc05::fence_after_sync();
-                        const uint32_t d = tm + x * S::TM_TILE + S::TM_S + b * N;
-                        const uint64_t ad = dq + (uint64_t)((x * S::Q_BYTES) >> 4);
-                        const uint64_t bd = dk + (uint64_t)((st * 2 * S::KV_BYTES) >> 4);
-                        // k-th 16-wide slice: +32 bytes inside a swizzle row, next half after 4
+            bool vz_seen = !need_vz;
+            auto qk = [&](int x, int i) {                    // S_x = Q_x K_i^T
+                const uint32_t d = tm + x * S::TM_TILE + S::TM_S;
+                const uint64_t ad = dq + (uint64_t)((x * S::Q_BYTES) >> 4);
+                const uint64_t bd = dk + (uint64_t)(((i % KST) * S::KV_BYTES) >> 4);
+                // k-th 16-wide slice: +32 bytes inside a swizzle row, next half after 4
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t qoff = ((k >> 2) * S::Q_HALF + (k & 3) * 32) >> 4;
-                            const uint32_t koff = ((k >> 2) * S::KV_HALF + (k & 3) * 32) >> 4;
-                            tc05::mma_ss(d, ad + qoff, bd + koff, idesc_qk, k > 0 ? 1u : 0u);
-                        }
-                        tc05::commit(bar_s(x, b));
-                    }
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t qoff = ((k >> 2) * S::Q_HALF + (k & 3) * 32) >> 4;
+                    const uint32_t koff = ((k >> 2) * S::KV_HALF + (k & 3) * 32) >> 4;
+                    tc05::mma_ss(d, ad + qoff, bd + koff, idesc_qk, k > 0 ? 1u : 0u);
                 }
-                if (ok && j >= 1) {                           // O_x += P_x V_{j-1}
-                    const int jj = j - 1, b = jj & 1, st = jj % ST;
-                    if (jj == nT - 1 && need_vz) ok = mbar_wait_bounded(bar_vz, 0, kWaitLimit);
-                    for (int x = 0; ok && x < 2; ++x) {
-                        if (jj >= nTx(x)) continue;
-                        if (!mbar_wait_bounded(bar_p(x, b), (jj >> 1) & 1, kWaitLimit)) {
-                            ok = false;
-                            break;
-                        }
-                        tc05::fence_after_sync();
-                        const uint32_t base = tm + x * S::TM_TILE;
-                        const uint64_t vd = dv + (uint64_t)((st * 2 * S::KV_BYTES) >> 4);
-                        // k-th 16 keys: 16 rows of 128 bytes further
+                tc05::commit(bar_s(x));
+            };
+            auto pv = [&](int x, int i) -> bool {            // O_x += P_x V_i
+                const int sv = i % VST;
+                if (!mbar_wait_bounded(bar_vfull(sv), (i / VST) & 1, kWaitLimit)) return false;
+                if (i == nT - 1 && !vz_seen) {
+                    if (!mbar_wait_bounded(bar_vz, 0, kWaitLimit)) return false;
+                    vz_seen = true;
+                }
+                if (!mbar_wait_bounded(bar_p(x), i & 1, kWaitLimit)) return false;
+                tc05::fence_after_sync();
+                const uint32_t base = tm + x * S::TM_TILE;
+                const uint64_t vd = dv + (uint64_t)((sv * S::KV_BYTES) >> 4);
+                // k-th 16 keys: 16 rows of 128 bytes further; P pairs 8 columns further
 #pragma unroll
-                        for (int k = 0; k < N / 16; ++k)
-                            tc05::mma_ts(base + S::TM_O, base + S::TM_S + b * N + 8 * k, vd + (uint64_t)(k * 128),
-                                         idesc_pv, (jj > 0 || k > 0) ? 1u : 0u);
-                        tc05::commit(bar_o(x, b));
-                    }
-                    if (ok) tc05::commit(bar_empty(st));
+                for (int k = 0; k < N / 16; ++k)
+                    tc05::mma_ts(base + S::TM_O, base + S::TM_S + 8 * k, vd + (uint64_t)(k * 128), idesc_pv,
+                                 (i > 0 || k > 0) ? 1u : 0u);
+                if (i == nTx(x) - 1) tc05::commit(bar_o(x));
+                return true;
+            };
+            for (int i = 0; ok && i < nT; ++i) {
+                if (!mbar_wait_bounded(bar_kfull(i % KST), (i / KST) & 1, kWaitLimit)) { ok = false; break; }
+                tc05::fence_after_sync();
+                if (i < nT0) qk(0, i);
+                if (two && i >= 1) {                         // V(i-1) last read by PV_1(i-1)
+                    if (!pv(1, i - 1)) { ok = false; break; }
+                    tc05::commit(bar_vempty((i - 1) % VST));
                 }
+                if (i < nT1) qk(1, i);
+                tc05::commit(bar_kempty(i % KST));
+                if (i < nT0) {
+                    if (!pv(0, i)) { ok = false; break; }
+                    if (!two) tc05::commit(bar_vempty(i % VST));
+                }
+            }
+            if (ok && two) {
+                if (pv(1, nT - 1)) tc05::commit(bar_vempty((nT - 1) % VST));
+                else ok = false;
             }
             if (!ok) flag_error(p.errors, PKV_DEVERR_WAIT);
             // every MMA issued above is complete before the tensor memory is freed
@@ -368,28 +383,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint32_t trow = tm + x * S::TM_TILE + ((uint32_t)(wq * 32) << 16);
             const float sl2 = p.scale_log2;
             float m_ref = -INFINITY, l = 0.f;           // reference max (log2 units), sum of weights
-            for (int j = 0; j < nTme; ++j) {
-                const int b = j & 1;
-                if (!warp_wait(bar_s(x, b), (j >> 1) & 1)) { ok = false; break; }
+            for (int i = 0; i < nTme; ++i) {
+                if (!warp_wait(bar_s(x), i & 1)) { ok = false; break; }
                 tc05::fence_after_sync();
-                uint32_t sv[64];
-                tc05::tmem_ld32(trow + S::TM_S + b * N, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                tc05::tmem_ld32(trow + S::TM_S + b * N + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                tc05::tmem_wait_ld();
-                const int key0 = j * N;
-                if (__any_sync(kAll, key0 + N - 1 > pos)) {      // a diagonal (or past-the-end) tile
+                const int key0 = i * N;
+                const bool diag = __any_sync(kAll, key0 + N - 1 > pos);   // a diagonal (or past-the-end) tile
+                // masked keys read as -inf (their logits may be NaN past the context end)
+                auto mask = [&](uint32_t (&v)[32], int col0) {
+                    if (diag) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (key0 + c > pos) sv[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 32; ++c)
+                            if (key0 + col0 + c > pos) v[c] = __float_as_uint(-INFINITY);
+                    }
+                };
+                // pass 1: the row maximum, 64 columns at a time
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int h = 0; h < N / 64; ++h) {
+                    uint32_t va[32], vb[32];
+                    tc05::tmem_ld32(trow + S::TM_S + 64 * h, va);
+                    tc05::tmem_ld32(trow + S::TM_S + 64 * h + 32, vb);
+                    tc05::tmem_wait_ld();
+                    mask(va, 64 * h);
+                    mask(vb, 64 * h + 32);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            m4[a] = max3(m4[a], __uint_as_float(va[c + a]), __uint_as_float(va[c + 4 + a]));
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            m4[a] = max3(m4[a], __uint_as_float(vb[c + a]), __uint_as_float(vb[c + 4 + a]));
                 }
-                float m4[4];
-#pragma unroll
-                for (int a = 0; a < 4; ++a) m4[a] = __uint_as_float(sv[a]);
-#pragma unroll
-                for (int c = 4; c < 64; c += 8)
-#pragma unroll
-                    for (int a = 0; a < 4; ++a)
-                        m4[a] = max3(m4[a], __uint_as_float(sv[c + a]), __uint_as_float(sv[c + 4 + a]));
                 const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float mt = mx * sl2;                  // the scale is positive
                 const bool raise = mt > m_ref + 8.f;
@@ -397,31 +424,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const float alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
                 const float neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
                 l *= alpha;
-                uint32_t pk[32];
-                const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
-                uint64_t lsum[4] = {0, 0, 0, 0};         // four packed partial sums (+0.0 bits)
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const uint64_t z = f2fma(f2pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])),
-                                             sl2x2, refx2);
-                    float z0, z1;
-                    f2unpack(z, z0, z1);
-                    const float p0 = ex2(z0), p1 = ex2(z1);
-                    lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
-                    pk[c] = Elem<T>::pack2(p0, p1);
-                }
-                {
-                    float a0, a1, b0, b1, c0, c1, d0, d1;
-                    f2unpack(lsum[0], a0, a1);
-                    f2unpack(lsum[1], b0, b1);
-                    f2unpack(lsum[2], c0, c1);
-                    f2unpack(lsum[3], d0, d1);
-                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-                }
-                // O holds PV of tiles < j: rescale rows whose reference moved (after PV(j-1) is done)
-                if (j >= 1 && __any_sync(kAll, alpha != 1.f)) {
-                    if (!warp_wait(bar_o(x, (j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
-                    tc05::fence_after_sync();
+                // O holds PV of tiles < i, complete (the S commit covers it): rescale
+                // rows whose reference moved
+                if (i >= 1 && __any_sync(kAll, alpha != 1.f)) {
 #pragma unroll
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t ov[32];
@@ -431,16 +436,50 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                         tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
                     }
-                    tc05::tmem_wait_st();
                 }
-                tc05::tmem_st32(trow + S::TM_S + b * N, pk);      // P over S (this row only)
+                // pass 2: weights, 32 keys (16 columns of P) at a time; the next
+                // chunk's load overlaps this chunk's arithmetic.  P chunk c lands
+                // on S columns 16c .. 16c+15, all read before (chunk c covers
+                // 32c .. 32c+31)
+                const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
+                uint64_t lsum[4] = {0, 0, 0, 0};         // four packed partial sums (+0.0 bits)
+                uint32_t buf[2][32];
+                tc05::tmem_ld32(trow + S::TM_S, buf[0]);
+                tc05::tmem_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < N / 32; ++ch) {
+                    uint32_t(&cur)[32] = buf[ch & 1];
+                    if (ch + 1 < N / 32) tc05::tmem_ld32(trow + S::TM_S + 32 * (ch + 1), buf[(ch + 1) & 1]);
+                    mask(cur, 32 * ch);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const uint64_t z = f2fma(f2pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
+                                                 sl2x2, refx2);
+                        float z0, z1;
+                        f2unpack(z, z0, z1);
+                        const float p0 = ex2(z0), p1 = ex2(z1);
+                        lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
+                        pk[c] = Elem<T>::pack2(p0, p1);
+                    }
+                    tc05::tmem_st16(trow + S::TM_S + 16 * ch, pk);   // P over S (this row only)
+                    tc05::tmem_wait_ld();
+                }
+                {
+                    float a0, a1, b0, b1, c0, c1, d0, d1;
+                    f2unpack(lsum[0], a0, a1);
+                    f2unpack(lsum[1], b0, b1);
+                    f2unpack(lsum[2], c0, c1);
+                    f2unpack(lsum[3], d0, d1);
+                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+                }
                 tc05::tmem_wait_st();
                 tc05::fence_before_sync();
-                mbar_arrive(bar_p(x, b));
+                mbar_arrive(bar_p(x));
                 m_ref = new_ref;
             }
             // ---- epilogue: O / l to the output ----
-            if (ok && warp_wait(bar_o(x, (nTme - 1) & 1), ((nTme - 1) >> 1) & 1)) {
+            if (ok && warp_wait(bar_o(x), 0)) {
                 tc05::fence_after_sync();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 T* orow = reinterpret_cast<T*>(p.out) +
