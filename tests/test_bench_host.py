@@ -90,3 +90,25 @@ def test_reference_arm_other_ranks_do_nothing():
     class A:
         workload = "tiny_mha_f32"
     assert bench.run_reference(A(), rank=1, world=2) is None
+
+
+def test_tensor_peak_follows_the_sampled_clock():
+    burst, kind, b2 = bench.tensor_peak({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})
+    assert "burst" in kind and burst == b2
+    sus, kind, b3 = bench.tensor_peak({"sm_mhz": 1300.0, "sm_max_mhz": 1965.0})
+    assert "sustained" in kind and sus <= b3
+    assert "burst" in bench.tensor_peak(None)[1]
+
+
+def test_prefill_flop_model():
+    """Causal pairs: every query i of n at position L - n + i sees L - n + i + 1 keys."""
+    lay = wl.make_prefill_layout(context_lens=[5, 300, 7], query_lens=[5, 17, 1], dtype="bf16",
+                                 num_heads=4, num_kv_heads=2, head_size=64, block_size=16)
+    brute = sum(L - n + i + 1 for L, n in [(5, 5), (300, 17), (7, 1)] for i in range(n))
+    assert wl.prefill_pairs(lay) == brute
+    assert bench.prefill_flops(lay) == 4 * 64 * 4 * brute
+    slots = bench.prefill_slots(lay)
+    assert len(slots) == 23
+    # the slot of sequence 1's last query is its last context position
+    L, bs = 300, 16
+    assert slots[5 + 16] == lay.block_tables[1, (L - 1) // bs] * bs + (L - 1) % bs
