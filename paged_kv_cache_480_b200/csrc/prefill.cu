@@ -5,49 +5,21 @@
 
 #include "prefill.cuh"
 #include "prefill_kernel.cuh"
+#include "tmap.cuh"
 
 namespace pkv {
 namespace {
 
 constexpr int kMaxDevices = 64;
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver's tensor-map encoder, looked up once through the runtime (the
-// library links no driver library).
-EncodeTiledFn encoder() {
-    static std::atomic<EncodeTiledFn> cached{nullptr};
-    EncodeTiledFn fn = cached.load(std::memory_order_acquire);
-    if (fn) return fn;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult found = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &found) != cudaSuccess ||
-        found != cudaDriverEntryPointSuccess || ptr == nullptr)
-        return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    cached.store(fn, std::memory_order_release);
-    return fn;
-}
-
-// Tiled map over a row-major tensor, innermost dimension first; boxes of
-// 64 elements (128 bytes) x ..., 128-byte swizzle, zero fill out of bounds.
-bool encode(EncodeTiledFn fn, CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base,
-            const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-    const cuuint32_t elem_strides[3] = {1, 1, 1};
-    return fn(map, type, (cuuint32_t)rank, const_cast<void*>(base), dims, strides_bytes, box,
-              elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+bool encode(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+    return encode_tiled(map, type, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <typename T, int D, int BS, int G>
 pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     using S = PrefillShape<T, D, BS, G>;
-    EncodeTiledFn fn = encoder();
-    if (!fn) return PKV_ERR_CUDA;
     const CUtensorMapDataType type =
         std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const cuuint64_t esz = sizeof(T);
@@ -56,7 +28,7 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
         const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.num_heads, (cuuint64_t)a.num_tokens};
         const cuuint64_t strides[2] = {D * esz, (cuuint64_t)a.num_heads * D * esz};
         const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)S::QT};
-        if (!encode(fn, &tm_q, type, 3, a.q, dims, strides, box)) return PKV_ERR_CUDA;
+        if (!encode(&tm_q, type, 3, a.q, dims, strides, box)) return PKV_ERR_CUDA;
     }
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
     if (rows > 0x7fffffff - BS) return PKV_ERR_UNSUPPORTED;
@@ -64,8 +36,8 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
         const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
         const cuuint64_t strides[1] = {D * esz};
         const cuuint32_t box[2] = {64, (cuuint32_t)BS};
-        if (!encode(fn, &tm_k, type, 2, a.k_cache, dims, strides, box)) return PKV_ERR_CUDA;
-        if (!encode(fn, &tm_v, type, 2, a.v_cache, dims, strides, box)) return PKV_ERR_CUDA;
+        if (!encode(&tm_k, type, 2, a.k_cache, dims, strides, box)) return PKV_ERR_CUDA;
+        if (!encode(&tm_v, type, 2, a.v_cache, dims, strides, box)) return PKV_ERR_CUDA;
     }
     PrefillParams p;
     std::memset(&p, 0, sizeof p);
