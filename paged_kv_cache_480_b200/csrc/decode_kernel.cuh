@@ -762,8 +762,18 @@ __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, cons
 // ===========================================================================
 // The kernel: prologue, producer (bulk-copy ring) and consumer loop.
 // ===========================================================================
+#ifndef PKV_FP8_THREADS
+#define PKV_FP8_THREADS 512
+#endif
+// Up to 12 consumer warps (16 over an FP8 cache, whose tiles are half the
+// size) per CTA; the host picks the count.
+template <typename TC>
+constexpr int decode_max_threads() {
+    return std::is_same<TC, fp8e4m3>::value ? PKV_FP8_THREADS : 384;
+}
+
 template <typename TQ, typename TC, int D, int BS, int G>
-__global__ void __launch_bounds__(384, 1) paged_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(decode_max_threads<TC>(), 1) paged_decode_kernel(const DecodeParams p) {
     using S = DecodeShape<TQ, TC, D, BS, G>;
     using L = WarpSmem<TQ, TC, D, BS, G>;
     constexpr bool kSameType = std::is_same<TQ, TC>::value;   // fused cache write needs it

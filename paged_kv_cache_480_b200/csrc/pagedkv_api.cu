@@ -9,6 +9,13 @@
 #include "pagedkv.h"
 #include "prefill.cuh"
 
+#ifndef PKV_FP8_WCAP
+#define PKV_FP8_WCAP 16
+#endif
+#ifndef PKV_FP8_RMAX
+#define PKV_FP8_RMAX 3
+#endif
+
 namespace {
 
 __device__ unsigned int g_device_errors;
@@ -221,18 +228,19 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     // gain nothing); a ring of two stages per warp then keeps enough bytes
     // in flight.  Use the deepest ring (up to 4) that still fits eight
     // warps, else fewer warps with two stages.
-    int R = 4;
+    // An FP8 cache halves the bytes per element, so each warp must retire
+    // blocks twice as fast: it gets more consumer warps (up to
+    // PKV_FP8_WCAP) and the ring depth that lets that many fit.
+    const int want = fp8_cache ? PKV_FP8_WCAP : 8;
+    int R = fp8_cache ? PKV_FP8_RMAX : 4;
     uint32_t per_warp = warp_smem(dtype, fp8_cache, head_size, block_size, G, R);
-    while (R > 2 && (pkv::kMaxDynSmem - seq_smem) / per_warp < 8) {
+    while (R > 2 && (pkv::kMaxDynSmem - seq_smem) / per_warp < (uint32_t)want) {
         --R;
         per_warp = warp_smem(dtype, fp8_cache, head_size, block_size, G, R);
     }
     int W = (int)((pkv::kMaxDynSmem - seq_smem) / per_warp);
-    // An FP8 cache halves the bytes per element, so each warp must retire
-    // blocks twice as fast: give it up to 12 consumer warps (measured: 8 -> 12
-    // warps is 1.25x; the 16-bit path gains nothing past 8).
-    const int w_cap = fp8_cache ? 12 : 8;
-    if (W > w_cap) W = w_cap;
+    if (W > want) W = want;
+    if (fp8_cache && 32 * W > PKV_FP8_THREADS) W = PKV_FP8_THREADS / 32;
     if (W < 1) return PKV_ERR_UNSUPPORTED;
 
     unsigned char* ws = static_cast<unsigned char*>(workspace);
