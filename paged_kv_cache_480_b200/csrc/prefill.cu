@@ -55,6 +55,16 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     p.max_blocks_per_seq = a.max_blocks_per_seq;
     p.q_tiles = (a.max_query_len + S::CQ - 1) / S::CQ;
     p.cache_rows = (int)rows;
+    // scheduling groups: as many (sequence, KV head) pairs as keep their K/V
+    // (at the longest possible context) within half of L2
+    {
+        int dev = 0, l2 = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        const double pair_bytes = (double)a.max_blocks_per_seq * BS * D * sizeof(T) * 2.0;
+        const double fit = (l2 / 2.0) / (pair_bytes > 1.0 ? pair_bytes : 1.0);
+        p.group = fit < 1.0 ? 1 : (fit > 4096.0 ? 4096 : (int)fit);
+    }
     const int64_t grid = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
     if (grid > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
     auto kernel = paged_prefill_kernel<T, D, BS, G>;

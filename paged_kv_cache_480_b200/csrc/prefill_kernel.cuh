@@ -107,6 +107,7 @@ struct PrefillParams {
     float scale_log2;                 // softmax scale * log2(e), > 0
     int num_tokens, num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq;
     int q_tiles;                      // CTAs (query-tile pairs) per (sequence, KV head)
+    int group;                        // (sequence, KV head) pairs per scheduling group, >= 1
     int cache_rows;                   // rows of the [NB * Hkv * bs][D] view of a cache
 };
 
@@ -168,8 +169,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- which queries: the later ones (more keys) are scheduled first ----
     const int Hkv = p.num_kv_heads;
     const int pairs = p.num_seqs * Hkv;
-    const int tile = p.q_tiles - 1 - (int)(blockIdx.x / pairs);
-    const int rest = blockIdx.x % pairs;
+// groups of p.group (sequence, KV head) pairs, one after the other; inside
+    // a group the tiles with most keys go first.  The host sizes groups so
+    // that a group's K/V fits in half of L2 while its query tiles read it.
+    const int gp = min(p.group, pairs);
+    const int per_group = gp * p.q_tiles;
+    const int grp = (int)blockIdx.x / per_group;
+    const int in_g = (int)blockIdx.x - grp * per_group;
+    const int g_pairs = min(gp, pairs - grp * gp);        // the last group may be smaller
+    const int tile = p.q_tiles - 1 - in_g / g_pairs;
+    const int rest = grp * gp + in_g % g_pairs;
     const int g = rest % Hkv;
     const int s = rest / Hkv;
     const int q0 = p.query_start_loc[s];
