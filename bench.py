@@ -42,10 +42,11 @@ def parse():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "prefill"],
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap", "prefill", "cache_ops"],
                     help="swap: swap_blocks between the GPU pool and a pinned host pool; "
                          "prefill: cache write + causal prefill attention (--workload "
-                         "prefill_llama7b_bf16 or chunked_gqa_bf16)")
+                         "prefill_llama7b_bf16 or chunked_gqa_bf16); cache_ops: reshape_and_cache and "
+                         "copy_blocks alone, GB/s of bytes read + written")
     ap.add_argument("--kv-cache", default="auto", choices=["auto", "fp8"],
                     help="fp8: E4M3 cache written by reshape_and_cache_fp8kv, read by the fp8 decode")
     ap.add_argument("--fused", action="store_true",
@@ -256,6 +257,27 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
+def prefill_source_sha():
+    h = hashlib.sha256()
+    for f in ("prefill_kernel.cuh", "prefill.cu", "tc05.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_480_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_prefill_traffic(workload):
+    """DRAM bytes per prefill launch from the committed ncu capture, if it
+    still matches the kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        e = json.load(f).get(workload)
+    if not e or e.get("source_sha") != prefill_source_sha():
+        return None
+    return e.get("bytes_per_call")
+
+
 def profiled_traffic(workload, block_size):
     """DRAM bytes per decode call from a committed ncu summary, if it still
     matches the kernel source (else None)."""
@@ -274,13 +296,13 @@ def profiled_traffic(workload, block_size):
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(lay, host, budget_s, max_seqs=None):
+def oracle_sample(lay, host, budget_s, max_seqs=None, threads=None):
     """Time the oracle on leading sequences of the workload (bounded), repeating
     until ~budget_s of work; returns (GB/s, seconds, bytes, seqs, threads)."""
     import oracle
     S = lay.num_seqs if max_seqs is None else min(max_seqs, lay.num_seqs)
     sub = lambda a: a[:S]
-    threads = oracle.default_threads()
+    threads = threads or oracle.default_threads()
     from paged_kv_cache_480_b200 import workloads as wl
     sublay = wl.Layout(**{**lay.__dict__, "num_seqs": S, "context_lens": sub(lay.context_lens),
                           "block_tables": sub(lay.block_tables), "slot_mapping": sub(lay.slot_mapping)})
@@ -490,9 +512,13 @@ def run_ours(args, rank, world, local_rank):
             host = host_arrays(ten, lay.dtype)
             gbs, t, b, seqs, threads = oracle_sample(lay, host, 10.0,
                                                      max_seqs=max(1, lay.num_seqs // 8))
+            gbs1, t1, _, seqs1, _ = oracle_sample(lay, host, 5.0, max_seqs=max(1, lay.num_seqs // 32), threads=1)
             result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                                       "sample": f"fp64 oracle over the first {max(1, lay.num_seqs // 8)} "
-                                                f"sequences, repeated: {seqs} sequence-passes in {t:.1f} s"}
+                                                f"sequences, repeated: {seqs} sequence-passes in {t:.1f} s",
+                                      "value_1core": gbs1,
+                                      "sample_1core": f"first {max(1, lay.num_seqs // 32)} sequences on one "
+                                                      f"thread: {seqs1} sequence-passes in {t1:.1f} s"}
     return result
 
 
@@ -733,7 +759,9 @@ def run_prefill(args, rank, world, local_rank):
                          "parallelism": f"replicas x{world}"},
               "roofline": {"kernel": "paged_attention_prefill", "bound": "tensor", "achieved": achieved,
                            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                           "frac_of_burst": achieved / burst, "traffic": None, "algorithmic_flops": flops,
+                           "frac_of_burst": achieved / burst, "traffic": profiled_prefill_traffic(lay.name),
+                           "traffic_note": "DRAM bytes per launch, one-pass ncu capture with a cold L2",
+                           "algorithmic_flops": flops,
                            "avg_call_us": k_avg * 1e3},
               "gpu_launches": 2 * args.steps, "clocks": clocks, "device_errors": errors}
     if not args.no_e2e:
@@ -851,6 +879,75 @@ def run_prefill_reference(args, rank, world):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_cache_ops(args, rank, world, local_rank):
+    """reshape_and_cache and copy_blocks timed alone, in GB/s of the bytes
+    they read and write (algorithmic: K and V rows and slots; source and
+    destination blocks).  L2 is flushed before every timed call (a 256 MB
+    write), each call timed with its own CUDA events."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    from paged_kv_cache_480_b200 import workloads as wl
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    pkv.load_library()
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3)
+        return statistics.median(ts)
+
+    lines = []
+
+    def line(metric, nbytes, t, cfg):
+        lines.append({"metric": metric, "value": nbytes / t / 1e9, "unit": "GB/s", "n_gpus": world,
+                      "steps": 20, "warmup": 3, "ms_per_step": t * 1e3, "higher_is_better": True,
+                      "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": cfg, "bytes": nbytes, "l2": "flushed before every call"},
+                      "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks()[0],
+                                   "unit": "GB/s", "frac": nbytes / t / 1e9 / peaks()[0],
+                                   "peak_kind": peaks()[1]},
+                      "gpu_launches": 20})
+
+    # reshape_and_cache: one decode step of the 7B-shaped workload, and a prefill's chunk
+    lay = wl.make_layout("llama7b_bf16")
+    ten = wl.make_tensors(lay, device=device)
+    sm = torch.from_numpy(lay.slot_mapping).to(device)
+    row = lay.num_kv_heads * lay.head_size * 2
+    t = timed(lambda: pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm,
+                                            stream=stream))
+    line("reshape_and_cache GB/s (read + write)", lay.num_seqs * (4 * row + 8), t,
+         f"llama7b_bf16 decode step: {lay.num_seqs} tokens x 32 heads x 128")
+    del ten
+    play, pten = prefill_workload("prefill_llama7b_bf16", device)
+    T = int(play.extra["query_start_loc"][-1])
+    t = timed(lambda: pkv.reshape_and_cache(pten["k_new"], pten["v_new"], pten["k_cache"], pten["v_cache"],
+                                            pten["slots"], stream=stream), reps=10)
+    line("reshape_and_cache GB/s (read + write)", T * (4 * row + 8), t,
+         f"prefill_llama7b_bf16 chunk write: {T} tokens x 32 heads x 128")
+    del pten
+    # copy_blocks: the first fork step of the parallel-sampling workload
+    lay, ten, pairs = build_cow_state(device)
+    pd = torch.from_numpy(np.ascontiguousarray(pairs)).to(device)
+    blk = lay.num_kv_heads * lay.block_size * lay.head_size * 2
+    t = timed(lambda: pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], pd, stream=stream))
+    line("copy_blocks GB/s (read + write)", len(pairs) * 2 * 2 * blk, t,
+         f"cow_bf16 first fork step: {len(pairs)} pairs x (K, V) x {blk // 1024} KB")
+    assert pkv.read_device_errors() == 0
+    return lines
+
+
 def run_swap(args, rank, world, local_rank):
     """swap_blocks throughput, device <-> pinned host, against a contiguous
     pinned copy of the same size measured in the same run (the host link's
@@ -928,8 +1025,9 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.measure == "swap":
-            for line in run_swap(args, rank, world, local_rank):
+        if args.measure in ("swap", "cache_ops"):
+            fn = run_swap if args.measure == "swap" else run_cache_ops
+            for line in fn(args, rank, world, local_rank):
                 if rank == 0:
                     print(json.dumps(line), flush=True)
             return
