@@ -388,7 +388,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const int r = wq * 32 + lane;               // row within the tile
             const int qi = i0 + x * S::QT + r / G;      // query of this row
             const bool valid = qi < n;
-            const int pos = valid ? L - n + qi : -1;    // keys 0 .. pos are visible
+            // keys 0 .. pos are visible.  Rows past the sequence's queries are
+            // never written and every row's softmax is its own, so they take no
+            // mask (a mask there would turn every tile of their warp diagonal)
+            const int pos = valid ? L - n + qi : 0x7fffffff;
             const uint32_t trow = tm + x * S::TM_TILE + ((uint32_t)(wq * 32) << 16);
             const float sl2 = p.scale_log2;
             float m_ref = -INFINITY, l = 0.f;           // reference max (log2 units), sum of weights
