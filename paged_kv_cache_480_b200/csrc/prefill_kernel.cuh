@@ -408,87 +408,108 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             if (key0 + col0 + c > pos) v[c] = __float_as_uint(-INFINITY);
                     }
                 };
-                // pass 1: the row maximum, 64 columns at a time
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int h = 0; h < N / 64; ++h) {
-                    uint32_t va[32], vb[32];
-                    tc05::tmem_ld32(trow + S::TM_S + 64 * h, va);
-                    tc05::tmem_ld32(trow + S::TM_S + 64 * h + 32, vb);
+                // weights P = 2^(S * scale*log2e + neg_ref), 32 keys (16 columns of P)
+                // at a time, the next chunk's load overlapping this chunk's
+                // arithmetic; P chunk c lands on S columns 16c .. 16c+15, all read
+                // before (chunk c covers 32c .. 32c+31).  Adds the weights to l_add
+                // and, with track, returns the row's largest exponent.
+                auto weights = [&](float neg_ref, float& l_add, bool track) -> float {
+                    const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
+                    uint64_t lsum[4] = {0, 0, 0, 0};     // four packed partial sums (+0.0 bits)
+                    float zmax = -INFINITY;
+                    uint32_t buf[2][32];
+                    tc05::tmem_ld32(trow + S::TM_S, buf[0]);
                     tc05::tmem_wait_ld();
-                    mask(va, 64 * h);
-                    mask(vb, 64 * h + 32);
 #pragma unroll
-                    for (int c = 0; c < 32; c += 8)
+                    for (int ch = 0; ch < N / 32; ++ch) {
+                        uint32_t(&cur)[32] = buf[ch & 1];
+                        if (ch + 1 < N / 32) tc05::tmem_ld32(trow + S::TM_S + 32 * (ch + 1), buf[(ch + 1) & 1]);
+                        mask(cur, 32 * ch);
+                        uint32_t pk[16];
 #pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            m4[a] = max3(m4[a], __uint_as_float(va[c + a]), __uint_as_float(va[c + 4 + a]));
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8)
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            m4[a] = max3(m4[a], __uint_as_float(vb[c + a]), __uint_as_float(vb[c + 4 + a]));
-                }
-                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                const float mt = mx * sl2;                  // the scale is positive
-                const bool raise = mt > m_ref + 8.f;
-                const float new_ref = raise ? mt : m_ref;
-                const float alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
-                const float neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
-                l *= alpha;
-                // O holds PV of tiles < i, complete (the S commit covers it): rescale
-                // rows whose reference moved
-                if (i >= 1 && __any_sync(kAll, alpha != 1.f)) {
-#pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t ov[32];
-                        tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
+                        for (int c = 0; c < 16; ++c) {
+                            const uint64_t z = f2fma(f2pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
+                                                     sl2x2, refx2);
+                            float z0, z1;
+                            f2unpack(z, z0, z1);
+                            if (track) zmax = max3(zmax, z0, z1);
+                            const float p0 = ex2(z0), p1 = ex2(z1);
+                            lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
+                            pk[c] = Elem<T>::pack2(p0, p1);
+                        }
+                        tc05::tmem_st16(trow + S::TM_S + 16 * ch, pk);   // P over S (this row only)
                         tc05::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
                     }
-                }
-                // pass 2: weights, 32 keys (16 columns of P) at a time; the next
-                // chunk's load overlaps this chunk's arithmetic.  P chunk c lands
-                // on S columns 16c .. 16c+15, all read before (chunk c covers
-                // 32c .. 32c+31)
-                const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
-                uint64_t lsum[4] = {0, 0, 0, 0};         // four packed partial sums (+0.0 bits)
-                uint32_t buf[2][32];
-                tc05::tmem_ld32(trow + S::TM_S, buf[0]);
-                tc05::tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < N / 32; ++ch) {
-                    uint32_t(&cur)[32] = buf[ch & 1];
-                    if (ch + 1 < N / 32) tc05::tmem_ld32(trow + S::TM_S + 32 * (ch + 1), buf[(ch + 1) & 1]);
-                    mask(cur, 32 * ch);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const uint64_t z = f2fma(f2pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
-                                                 sl2x2, refx2);
-                        float z0, z1;
-                        f2unpack(z, z0, z1);
-                        const float p0 = ex2(z0), p1 = ex2(z1);
-                        lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
-                        pk[c] = Elem<T>::pack2(p0, p1);
-                    }
-                    tc05::tmem_st16(trow + S::TM_S + 16 * ch, pk);   // P over S (this row only)
-                    tc05::tmem_wait_ld();
-                }
-                {
                     float a0, a1, b0, b1, c0, c1, d0, d1;
                     f2unpack(lsum[0], a0, a1);
                     f2unpack(lsum[1], b0, b1);
                     f2unpack(lsum[2], c0, c1);
                     f2unpack(lsum[3], d0, d1);
-                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+                    l_add = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+                    return zmax;
+                };
+                // Once a row has a reference, most tiles do not raise it: take the
+                // weights at the current reference in one pass and keep them unless
+                // some row of the warp saw a logit more than 8 above its reference;
+                // then (and on a row's first tile) find the row maximum first.
+                bool two_pass = !__all_sync(kAll, m_ref != -INFINITY);
+                float neg_ref = -m_ref, alpha = 1.f;
+                for (int attempt = 0; attempt < 2; ++attempt) {
+                    if (two_pass) {
+                        // pass 1: the row maximum, 64 columns at a time
+                        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                        for (int h = 0; h < N / 64; ++h) {
+                            uint32_t va[32], vb[32];
+                            tc05::tmem_ld32(trow + S::TM_S + 64 * h, va);
+                            tc05::tmem_ld32(trow + S::TM_S + 64 * h + 32, vb);
+                            tc05::tmem_wait_ld();
+                            mask(va, 64 * h);
+                            mask(vb, 64 * h + 32);
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                                for (int a = 0; a < 4; ++a)
+                                    m4[a] = max3(m4[a], __uint_as_float(va[c + a]), __uint_as_float(va[c + 4 + a]));
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                                for (int a = 0; a < 4; ++a)
+                                    m4[a] = max3(m4[a], __uint_as_float(vb[c + a]), __uint_as_float(vb[c + 4 + a]));
+                        }
+                        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                        const float mt = mx * sl2;              // the scale is positive
+                        const bool raise = mt > m_ref + 8.f;
+                        const float new_ref = raise ? mt : m_ref;
+                        alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
+                        neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
+                        m_ref = new_ref;
+                        // O holds PV of tiles < i, complete (the S commit covers it):
+                        // rescale rows whose reference moved
+                        if (i >= 1 && __any_sync(kAll, alpha != 1.f)) {
+#pragma unroll
+                            for (int cc = 0; cc < D / 32; ++cc) {
+                                uint32_t ov[32];
+                                tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
+                                tc05::tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                                tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
+                            }
+                        }
+                    }
+                    float l_add;
+                    const float zmax = weights(neg_ref, l_add, !two_pass);
+                    if (!two_pass && __any_sync(kAll, zmax > 8.f)) {
+                        two_pass = true;                        // redo this tile
+                        continue;
+                    }
+                    l = l * alpha + l_add;
+                    break;
                 }
                 tc05::tmem_wait_st();
                 tc05::fence_before_sync();
                 mbar_arrive(bar_p(x));
-                m_ref = new_ref;
             }
             // ---- epilogue: O / l to the output ----
             if (ok && warp_wait(bar_o(x), 0)) {
