@@ -1,5 +1,6 @@
 /*
- * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache library: decode
+ * attention, cache maintenance and causal prefill over the paged cache.
  *
  * The library implements the data-parallel hot path of PagedAttention as
  * the pages describe it:
