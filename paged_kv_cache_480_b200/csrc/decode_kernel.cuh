@@ -136,6 +136,7 @@ constexpr unsigned kFull = 0xffffffffu;
 // ===========================================================================
 template <typename TQ, typename TC, int D, int BS, int G>
 struct FmaConsumer {
+    static constexpr bool kPairs = false;   // one block per consumer step
     using S = DecodeShape<TQ, TC, D, BS, G>;
     static constexpr int EPC = S::EPC;
     static constexpr int EPQ = Elem<TQ>::kPerChunk;  // q / out elements per 16-byte chunk
@@ -289,6 +290,7 @@ struct FmaConsumer {
 // ===========================================================================
 template <typename T, int D, int BS, int G>
 struct MmaConsumer {
+    static constexpr bool kPairs = false;   // one block per consumer step
     using S = DecodeShape<T, T, D, BS, G>;
     static_assert(sizeof(T) == 2, "tensor-core consumer needs 16-bit elements");
     static_assert(G <= 8, "the 8 MMA columns hold the query heads of one group");
@@ -573,11 +575,10 @@ struct MmaConsumerFp8 {
         l0 = l1 = 0.f;
     }
 
-    __device__ __forceinline__ void slice(const unsigned char* Kt, const unsigned char* Vt,
-                                          int nvalid, float scale_log2) {
+    // S^T of one 16-token slice: sc = K[16 x D] . Q^T (D/16 MMAs)
+    __device__ __forceinline__ void qk(const unsigned char* Kt, float (&sc)[4]) const {
         const uint4* k0 = reinterpret_cast<const uint4*>(Kt + r * S::ROW);
         const uint4* k8 = reinterpret_cast<const uint4*>(Kt + (r + 8) * S::ROW);
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < KJ; ++j) {
             const uint4 a = k0[4 * j + c];
@@ -590,25 +591,49 @@ struct MmaConsumerFp8 {
                     e4m3x2_to_f16x2((uint16_t)(wa[hf] >> 16)), e4m3x2_to_f16x2((uint16_t)(wb[hf] >> 16)),
                     qf[j][2 * hf], qf[j][2 * hf + 1]);
         }
+    }
+
+    // Logits of a slice in log2 units; tokens at or past nvalid are -inf.
+    __device__ __forceinline__ void logits(const float (&sc)[4], int nvalid, float scale_log2,
+                                           float (&z)[4]) const {
         const bool v0 = r < nvalid, v8 = r + 8 < nvalid;
-        const float z0 = v0 ? sc[0] * scale_log2 : -INFINITY;
-        const float z1 = v0 ? sc[1] * scale_log2 : -INFINITY;
-        const float z2 = v8 ? sc[2] * scale_log2 : -INFINITY;
-        const float z3 = v8 ? sc[3] * scale_log2 : -INFINITY;
-        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+        z[0] = v0 ? sc[0] * scale_log2 : -INFINITY;
+        z[1] = v0 ? sc[1] * scale_log2 : -INFINITY;
+        z[2] = v8 ? sc[2] * scale_log2 : -INFINITY;
+        z[3] = v8 ? sc[3] * scale_log2 : -INFINITY;
+    }
+
+    // Weights of a slice against the new maxima (fp16 pairs), added to l, and
+    // moved to the B-fragment layout of the PV products.
+    __device__ __forceinline__ void weights(const float (&z)[4], float n0, float n1, float& s0, float& s1,
+                                            uint32_t& pb0, uint32_t& pb1) const {
+        const uint32_t pk_lo = Elem<__half>::pack2(ex2(z[0] - n0), ex2(z[1] - n1));
+        const uint32_t pk_hi = Elem<__half>::pack2(ex2(z[2] - n0), ex2(z[3] - n1));
+        s0 += lo_f(pk_lo) + lo_f(pk_hi);
+        s1 += hi_f(pk_lo) + hi_f(pk_hi);
+        const int src0 = (2 * c) * 4 + (r >> 1), src1 = src0 + 4;
+        const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+        const uint32_t x0 = __shfl_sync(kFull, pk_lo, src0), x1 = __shfl_sync(kFull, pk_lo, src1);
+        const uint32_t y0 = __shfl_sync(kFull, pk_hi, src0), y1 = __shfl_sync(kFull, pk_hi, src1);
+        pb0 = prmt(x0, x1, sel);
+        pb1 = prmt(y0, y1, sel);
+    }
+
+    // New running maxima from a slice's (or two slices') row maxima; rescales
+    // l and the accumulator.  Returns the maxima to take weights against.
+    __device__ __forceinline__ void update_max(float mx0, float mx1, float& n0, float& n1) {
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
             mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
             mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
         }
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        n0 = fmaxf(m0, mx0);
+        n1 = fmaxf(m1, mx1);
         const float al0 = ex2(m0 - n0), al1 = ex2(m1 - n1);
         m0 = n0;
         m1 = n1;
-        const uint32_t pk_lo = Elem<__half>::pack2(ex2(z0 - n0), ex2(z1 - n1));
-        const uint32_t pk_hi = Elem<__half>::pack2(ex2(z2 - n0), ex2(z3 - n1));
-        l0 = l0 * al0 + lo_f(pk_lo) + lo_f(pk_hi);
-        l1 = l1 * al1 + hi_f(pk_lo) + hi_f(pk_hi);
+        l0 *= al0;
+        l1 *= al1;
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             o[m][0] *= al0;
@@ -616,11 +641,10 @@ struct MmaConsumerFp8 {
             o[m][1] *= al1;
             o[m][3] *= al1;
         }
-        const int src0 = (2 * c) * 4 + (r >> 1), src1 = src0 + 4;
-        const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
-        const uint32_t x0 = __shfl_sync(kFull, pk_lo, src0), x1 = __shfl_sync(kFull, pk_lo, src1);
-        const uint32_t y0 = __shfl_sync(kFull, pk_hi, src0), y1 = __shfl_sync(kFull, pk_hi, src1);
-        const uint32_t pb0 = prmt(x0, x1, sel), pb1 = prmt(y0, y1, sel);
+    }
+
+    // O^T += V^T[D x 16 tok] . P^T (D/16 MMAs)
+    __device__ __forceinline__ void pv(const unsigned char* Vt, int nvalid, uint32_t pb0, uint32_t pb1) {
         // V rows 2c, 2c+1, 2c+8, 2c+9: bytes = dims r*D/8 .. +D/8
         uint32_t w[4][VB / 4];
         const int rows[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
@@ -650,14 +674,65 @@ struct MmaConsumerFp8 {
         }
     }
 
+    __device__ __forceinline__ void slice(const unsigned char* Kt, const unsigned char* Vt,
+                                          int nvalid, float scale_log2) {
+        float sc[4] = {0.f, 0.f, 0.f, 0.f}, z[4];
+        qk(Kt, sc);
+        logits(sc, nvalid, scale_log2, z);
+        float n0, n1;
+        update_max(fmaxf(z[0], z[2]), fmaxf(z[1], z[3]), n0, n1);
+        uint32_t pb0, pb1;
+        weights(z, n0, n1, l0, l1, pb0, pb1);
+        pv(Vt, nvalid, pb0, pb1);
+    }
+
+    // Two 16-token slices of one item with one softmax update: the two
+    // independent QK and PV chains overlap, halving the per-token latency
+    // of the warp.
+    __device__ __forceinline__ void slice2(const unsigned char* Ka, const unsigned char* Va, int nva,
+                                           const unsigned char* Kb, const unsigned char* Vb, int nvb,
+                                           float scale_log2) {
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f}, za[4], zb[4];
+        qk(Ka, sa);
+        qk(Kb, sb);
+        logits(sa, nva, scale_log2, za);
+        logits(sb, nvb, scale_log2, zb);
+        float n0, n1;
+        update_max(fmaxf(fmaxf(za[0], za[2]), fmaxf(zb[0], zb[2])), fmaxf(fmaxf(za[1], za[3]), fmaxf(zb[1], zb[3])),
+                   n0, n1);
+        uint32_t pa0, pa1, pb0, pb1;
+        weights(za, n0, n1, l0, l1, pa0, pa1);
+        weights(zb, n0, n1, l0, l1, pb0, pb1);
+        pv(Va, nva, pa0, pa1);
+        pv(Vb, nvb, pb0, pb1);
+    }
+
+    // Pairs of blocks of one item are handed to block2 (block size 16: one
+    // slice each); a 32-token block is a pair of slices itself.  With 8
+    // query heads the MMA columns are full and the pair's extra registers
+    // cost more than the overlap gains (measured), so G = 8 takes one slice
+    // at a time.
+    static constexpr bool kPairSlices = G < 8;
+    static constexpr bool kPairs = BS == 16 && kPairSlices;
+
     __device__ __forceinline__ void block(const unsigned char* Kt, const unsigned char* Vt,
                                           int nvalid, float scale_log2) {
+        if (BS == 32 && kPairSlices && nvalid > 16) {
+            slice2(Kt, Vt, 16, Kt + 16 * S::ROW, Vt + 16 * S::ROW, nvalid - 16, scale_log2);
+            return;
+        }
 #pragma unroll
         for (int sl = 0; sl < BS / 16; ++sl) {
             const int nv = nvalid - 16 * sl;
             if (nv <= 0) break;
             slice(Kt + sl * 16 * S::ROW, Vt + sl * 16 * S::ROW, nv, scale_log2);
         }
+    }
+
+    __device__ __forceinline__ void block2(const unsigned char* Ka, const unsigned char* Va, int nva,
+                                           const unsigned char* Kb, const unsigned char* Vb, int nvb,
+                                           float scale_log2) {
+        slice2(Ka, Va, nva, Kb, Vb, nvb, scale_log2);
     }
 
     __device__ __forceinline__ void finish(const StageMeta& mt, const DecodeParams& p) {
@@ -765,15 +840,15 @@ __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, cons
 #ifndef PKV_FP8_THREADS
 #define PKV_FP8_THREADS 512
 #endif
-// Up to 12 consumer warps (16 over an FP8 cache, whose tiles are half the
-// size) per CTA; the host picks the count.
-template <typename TC>
+// Up to 12 consumer warps (16 for the tensor-core consumer over an FP8
+// cache, whose tiles are half the size) per CTA; the host picks the count.
+template <typename TQ, typename TC, int G>
 constexpr int decode_max_threads() {
-    return std::is_same<TC, fp8e4m3>::value ? PKV_FP8_THREADS : 384;
+    return (std::is_same<TC, fp8e4m3>::value && UseMma<TQ, TC, G>::value) ? PKV_FP8_THREADS : 384;
 }
 
 template <typename TQ, typename TC, int D, int BS, int G>
-__global__ void __launch_bounds__(decode_max_threads<TC>(), 1) paged_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_decode_kernel(const DecodeParams p) {
     using S = DecodeShape<TQ, TC, D, BS, G>;
     using L = WarpSmem<TQ, TC, D, BS, G>;
     constexpr bool kSameType = std::is_same<TQ, TC>::value;   // fused cache write needs it
@@ -959,6 +1034,34 @@ __global__ void __launch_bounds__(decode_max_threads<TC>(), 1) paged_decode_kern
         }
         const StageMeta mt = meta[cons_st];
         if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, qscale);
+        using Cons = ConsumerFor<TQ, TC, D, BS, G>;
+        if constexpr (Cons::kPairs) {
+            // the item's next block is in the next stage: take both together
+            if (!(mt.flags & kLast) && mt.nvalid > 0 && mt.newrow < 0 && consumed + 1 < issued) {
+                const int st2 = (cons_st + 1 == R) ? 0 : cons_st + 1;
+                const uint32_t ph2 = (cons_st + 1 == R) ? (phase ^ 1u) : phase;
+                if (!mbar_wait_bounded(bar0 + 8 * st2, ph2, kWaitLimit)) {
+                    flag_error(p.errors, PKV_DEVERR_WAIT);
+                    lost = true;
+                    break;
+                }
+                const StageMeta mt2 = meta[st2];
+                if (mt2.nvalid > 0 && mt2.newrow < 0) {
+                    const unsigned char* Ka = ring + (size_t)cons_st * 2 * S::TILE;
+                    const unsigned char* Kb = ring + (size_t)st2 * 2 * S::TILE;
+                    cons.block2(Ka, Ka + S::TILE, mt.nvalid, Kb, Kb + S::TILE, mt2.nvalid, qscale);
+                    if (mt2.flags & kLast) cons.finish(mt2, p);
+                    __syncwarp();
+                    consumed += 2;
+                    cons_st = st2;
+                    phase = ph2;
+                    if (++cons_st == R) { cons_st = 0; phase ^= 1u; }
+                    issue();
+                    issue();
+                    continue;
+                }
+            }
+        }
         if (mt.newrow >= 0) {
             // Fused cache write: put the new token's K and V rows into the tile
             // (it holds the slot's old bytes) and into the cache slot.

@@ -231,8 +231,11 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     // An FP8 cache halves the bytes per element, so each warp must retire
     // blocks twice as fast: it gets more consumer warps (up to
     // PKV_FP8_WCAP) and the ring depth that lets that many fit.
-    const int want = fp8_cache ? PKV_FP8_WCAP : 8;
-    int R = fp8_cache ? PKV_FP8_RMAX : 4;
+    // (the FP8 tensor-core consumer serves 16-bit q; fp32 q over an FP8
+    // cache takes the fp32 consumer with up to 12 warps)
+    const bool fp8_mma = fp8_cache && dtype != PKV_F32;
+    const int want = fp8_mma ? PKV_FP8_WCAP : (fp8_cache ? 12 : 8);
+    int R = fp8_mma ? PKV_FP8_RMAX : 4;
     uint32_t per_warp = warp_smem(dtype, fp8_cache, head_size, block_size, G, R);
     while (R > 2 && (pkv::kMaxDynSmem - seq_smem) / per_warp < (uint32_t)want) {
         --R;
@@ -240,7 +243,7 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     }
     int W = (int)((pkv::kMaxDynSmem - seq_smem) / per_warp);
     if (W > want) W = want;
-    if (fp8_cache && 32 * W > PKV_FP8_THREADS) W = PKV_FP8_THREADS / 32;
+    if (fp8_mma && 32 * W > PKV_FP8_THREADS) W = PKV_FP8_THREADS / 32;
     if (W < 1) return PKV_ERR_UNSUPPORTED;
 
     unsigned char* ws = static_cast<unsigned char*>(workspace);
