@@ -408,15 +408,152 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             if (key0 + col0 + c > pos) v[c] = __float_as_uint(-INFINITY);
                     }
                 };
-                // weights P = 2^(S * scale*log2e + neg_ref), 32 keys (16 columns of P)
-                // at a time, the next chunk's load overlapping this chunk's
-                // arithmetic; P chunk c lands on S columns 16c .. 16c+15, all read
-                // before (chunk c covers 32c .. 32c+31).  Adds the weights to l_add
-                // and, with track, returns the row's largest exponent.
-                auto weights = [&](float neg_ref, float& l_add, bool track) -> float {
-                    const uint64_t sl2x2 = f2pack(sl2, sl2), refx2 = f2pack(neg_ref, neg_ref);
-                    uint64_t lsum[4] = {0, 0, 0, 0};     // four packed partial sums (+0.0 bits)
-                    float zmax = -INFINITY;
+                // The weights of one 32-key chunk of S (16 columns of P):
+                // P = 2^(S * scale*log2e + neg_ref), summed into lsum.
+                auto chunk_w = [&](const uint32_t(&cur)[32], uint64_t refx2, uint64_t(&lsum)[4], uint32_t(&pk)[16]) {
+                    const uint64_t sl2x2 = f2pack(sl2, sl2);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const uint64_t z = f2fma(f2pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
+                                                 sl2x2, refx2);
+                        float z0, z1;
+                        f2unpack(z, z0, z1);
+                        const float p0 = ex2(z0), p1 = ex2(z1);
+                        lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
+                        pk[c] = Elem<T>::pack2(p0, p1);
+                    }
+                };
+                auto chunk_max = [&](const uint32_t(&cur)[32]) -> float {
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            m4[a] = max3(m4[a], __uint_as_float(cur[c + a]), __uint_as_float(cur[c + 4 + a]));
+                    return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                };
+                auto lsum_total = [&](const uint64_t(&lsum)[4]) -> float {
+                    float a0, a1, b0f, b1f, c0f, c1f, d0, d1;
+                    f2unpack(lsum[0], a0, a1);
+                    f2unpack(lsum[1], b0f, b1f);
+                    f2unpack(lsum[2], c0f, c1f);
+                    f2unpack(lsum[3], d0, d1);
+                    return ((a0 + a1) + (b0f + b1f)) + ((c0f + c1f) + (d0 + d1));
+                };
+                // O holds PV of the tiles before this one, complete (the S commit
+                // covers it): scale the rows whose reference moved
+                auto rescale_o = [&](float a) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t ov[32];
+                        tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
+                        tc05::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
+                        tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
+                    }
+                };
+                static_assert(N == 128, "four 32-key chunks per tile");
+                // P chunk c lands on S columns 16c .. 16c+15, so storing P chunks 0-3
+                // overwrites S chunks 0 and 1 only; S chunks 2 and 3 stay intact.
+                float l_add = 0.f, alpha = 1.f;
+                bool full = !__all_sync(kAll, m_ref != -INFINITY);
+                if (!full) {
+                    // Most tiles keep every row's reference: one sweep at it.  The P
+                    // of chunks 0 and 1 is held until no row of the warp has a logit
+                    // more than 8 above its reference there (else the tile is redone
+                    // from the intact S); chunks 2 and 3 are stored at once and
+                    // checked after, their S still intact for a recomputation.
+                    const uint64_t refx2 = f2pack(-m_ref, -m_ref);
+                    uint64_t lA[4] = {0, 0, 0, 0}, lB[4] = {0, 0, 0, 0};
+                    uint32_t b0[32], b1[32], pk0[16], pk1[16];
+                    tc05::tmem_ld32(trow + S::TM_S, b0);
+                    tc05::tmem_ld32(trow + S::TM_S + 32, b1);
+                    tc05::tmem_wait_ld();
+                    mask(b0, 0);
+                    mask(b1, 32);
+                    const float cmA = fmaxf(chunk_max(b0), chunk_max(b1));
+                    chunk_w(b0, refx2, lA, pk0);
+                    chunk_w(b1, refx2, lA, pk1);
+                    tc05::tmem_ld32(trow + S::TM_S + 64, b0);
+                    tc05::tmem_ld32(trow + S::TM_S + 96, b1);
+                    if (__any_sync(kAll, cmA * sl2 - m_ref > 8.f)) {
+                        tc05::tmem_wait_ld();
+                        full = true;                            // nothing stored: redo from S
+                    } else {
+                        tc05::tmem_st16(trow + S::TM_S, pk0);
+                        tc05::tmem_st16(trow + S::TM_S + 16, pk1);
+                        tc05::tmem_wait_ld();
+                        mask(b0, 64);
+                        mask(b1, 96);
+                        const float cmB = fmaxf(chunk_max(b0), chunk_max(b1));
+                        chunk_w(b0, refx2, lB, pk0);
+                        tc05::tmem_st16(trow + S::TM_S + 32, pk0);
+                        chunk_w(b1, refx2, lB, pk1);
+                        tc05::tmem_st16(trow + S::TM_S + 48, pk1);
+                        if (!__any_sync(kAll, cmB * sl2 - m_ref > 8.f)) {
+                            l_add = lsum_total(lA) + lsum_total(lB);
+                        } else {
+                            // a logit of chunk 2 or 3 rose more than 8 above its row's
+                            // reference: move to the row maximum, rescale the P of
+                            // chunks 0 and 1 and O, recompute chunks 2 and 3
+                            const float mt = fmaxf(cmA, cmB) * sl2;
+                            const bool raise = mt > m_ref + 8.f;
+                            const float new_ref = raise ? mt : m_ref;
+                            alpha = raise ? ex2(m_ref - new_ref) : 1.f;
+                            m_ref = new_ref;
+                            tc05::tmem_wait_st();
+                            if (__any_sync(kAll, alpha != 1.f)) {
+#pragma unroll
+                                for (int ch = 0; ch < 2; ++ch) {
+                                    uint32_t pv16[16];
+                                    tc05::tmem_ld16(trow + S::TM_S + 16 * ch, pv16);
+                                    tc05::tmem_wait_ld();
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) {
+                                        float lo, hi;
+                                        Elem<T>::widen2(pv16[e], lo, hi);
+                                        pv16[e] = Elem<T>::pack2(lo * alpha, hi * alpha);
+                                    }
+                                    tc05::tmem_st16(trow + S::TM_S + 16 * ch, pv16);
+                                }
+                                if (i >= 1) rescale_o(alpha);
+                            }
+                            const uint64_t ref2 = f2pack(-m_ref, -m_ref);
+                            uint64_t lC[4] = {0, 0, 0, 0};
+                            chunk_w(b0, ref2, lC, pk0);
+                            tc05::tmem_st16(trow + S::TM_S + 32, pk0);
+                            chunk_w(b1, ref2, lC, pk1);
+                            tc05::tmem_st16(trow + S::TM_S + 48, pk1);
+                            l_add = lsum_total(lA) * alpha + lsum_total(lC);
+                        }
+                    }
+                }
+                if (full) {
+                    // a row's first tile (or rows that have seen only masked keys, or
+                    // a jump in chunk 0 or 1): the row maximum first
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int hh = 0; hh < N / 64; ++hh) {
+                        uint32_t va[32], vb[32];
+                        tc05::tmem_ld32(trow + S::TM_S + 64 * hh, va);
+                        tc05::tmem_ld32(trow + S::TM_S + 64 * hh + 32, vb);
+                        tc05::tmem_wait_ld();
+                        mask(va, 64 * hh);
+                        mask(vb, 64 * hh + 32);
+                        mx = fmaxf(mx, fmaxf(chunk_max(va), chunk_max(vb)));
+                    }
+                    const float mt = mx * sl2;                  // the scale is positive
+                    const bool raise = mt > m_ref + 8.f;
+                    const float new_ref = raise ? mt : m_ref;
+                    alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
+                    m_ref = new_ref;
+                    if (i >= 1 && __any_sync(kAll, alpha != 1.f)) rescale_o(alpha);
+                    // weights at the new reference, the next chunk's load overlapping
+                    // this chunk's arithmetic (P chunk c lands on S columns already read)
+                    const float nr = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
+                    const uint64_t refx2 = f2pack(nr, nr);
+                    uint64_t lsum[4] = {0, 0, 0, 0};
                     uint32_t buf[2][32];
                     tc05::tmem_ld32(trow + S::TM_S, buf[0]);
                     tc05::tmem_wait_ld();
@@ -426,87 +563,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         if (ch + 1 < N / 32) tc05::tmem_ld32(trow + S::TM_S + 32 * (ch + 1), buf[(ch + 1) & 1]);
                         mask(cur, 32 * ch);
                         uint32_t pk[16];
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const uint64_t z = f2fma(f2pack(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
-                                                     sl2x2, refx2);
-                            float z0, z1;
-                            f2unpack(z, z0, z1);
-                            if (track) zmax = max3(zmax, z0, z1);
-                            const float p0 = ex2(z0), p1 = ex2(z1);
-                            lsum[c & 3] = f2add(lsum[c & 3], f2pack(p0, p1));
-                            pk[c] = Elem<T>::pack2(p0, p1);
-                        }
-                        tc05::tmem_st16(trow + S::TM_S + 16 * ch, pk);   // P over S (this row only)
+                        chunk_w(cur, refx2, lsum, pk);
+                        tc05::tmem_st16(trow + S::TM_S + 16 * ch, pk);
                         tc05::tmem_wait_ld();
                     }
-                    float a0, a1, b0, b1, c0, c1, d0, d1;
-                    f2unpack(lsum[0], a0, a1);
-                    f2unpack(lsum[1], b0, b1);
-                    f2unpack(lsum[2], c0, c1);
-                    f2unpack(lsum[3], d0, d1);
-                    l_add = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-                    return zmax;
-                };
-                // Once a row has a reference, most tiles do not raise it: take the
-                // weights at the current reference in one pass and keep them unless
-                // some row of the warp saw a logit more than 8 above its reference;
-                // then (and on a row's first tile) find the row maximum first.
-                bool two_pass = !__all_sync(kAll, m_ref != -INFINITY);
-                float neg_ref = -m_ref, alpha = 1.f;
-                for (int attempt = 0; attempt < 2; ++attempt) {
-                    if (two_pass) {
-                        // pass 1: the row maximum, 64 columns at a time
-                        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                        for (int h = 0; h < N / 64; ++h) {
-                            uint32_t va[32], vb[32];
-                            tc05::tmem_ld32(trow + S::TM_S + 64 * h, va);
-                            tc05::tmem_ld32(trow + S::TM_S + 64 * h + 32, vb);
-                            tc05::tmem_wait_ld();
-                            mask(va, 64 * h);
-                            mask(vb, 64 * h + 32);
-#pragma unroll
-                            for (int c = 0; c < 32; c += 8)
-#pragma unroll
-                                for (int a = 0; a < 4; ++a)
-                                    m4[a] = max3(m4[a], __uint_as_float(va[c + a]), __uint_as_float(va[c + 4 + a]));
-#pragma unroll
-                            for (int c = 0; c < 32; c += 8)
-#pragma unroll
-                                for (int a = 0; a < 4; ++a)
-                                    m4[a] = max3(m4[a], __uint_as_float(vb[c + a]), __uint_as_float(vb[c + 4 + a]));
-                        }
-                        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                        const float mt = mx * sl2;              // the scale is positive
-                        const bool raise = mt > m_ref + 8.f;
-                        const float new_ref = raise ? mt : m_ref;
-                        alpha = (raise && m_ref != -INFINITY) ? ex2(m_ref - new_ref) : 1.f;
-                        neg_ref = new_ref == -INFINITY ? 0.f : -new_ref;   // rows that see nothing yet
-                        m_ref = new_ref;
-                        // O holds PV of tiles < i, complete (the S commit covers it):
-                        // rescale rows whose reference moved
-                        if (i >= 1 && __any_sync(kAll, alpha != 1.f)) {
-#pragma unroll
-                            for (int cc = 0; cc < D / 32; ++cc) {
-                                uint32_t ov[32];
-                                tc05::tmem_ld32(trow + S::TM_O + cc * 32, ov);
-                                tc05::tmem_wait_ld();
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                                tc05::tmem_st32(trow + S::TM_O + cc * 32, ov);
-                            }
-                        }
-                    }
-                    float l_add;
-                    const float zmax = weights(neg_ref, l_add, !two_pass);
-                    if (!two_pass && __any_sync(kAll, zmax > 8.f)) {
-                        two_pass = true;                        // redo this tile
-                        continue;
-                    }
-                    l = l * alpha + l_add;
-                    break;
+                    l_add = lsum_total(lsum);
                 }
+                l = l * alpha + l_add;
                 tc05::tmem_wait_st();
                 tc05::fence_before_sync();
                 mbar_arrive(bar_p(x));

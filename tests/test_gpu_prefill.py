@@ -143,6 +143,57 @@ def test_prefill_rejects_f32_and_bad_shapes():
                                     bt, cl, qsl, lay.scale, max_query_len=31)
 
 
+JUMPS = [
+    # dtype, H, Hkv, D, bs, context lens, query lens
+    ("bf16", 8, 8, 128, 16, [700, 390], [700, 200]),
+    ("f16", 16, 2, 64, 32, [600, 333], [300, 333]),
+    ("bf16", 16, 4, 128, 32, [900], [260]),
+]
+
+
+@pytest.mark.parametrize("dtype,H,Hkv,D,bs,lens,nq", JUMPS)
+def test_prefill_logit_jumps(dtype, H, Hkv, D, bs, lens, nq):
+    """Keys scaled by 8 at random positions past the first key tile: their
+    logits rise far above everything a row saw before, anywhere inside a key
+    tile, so the row's reference moves in the middle of a tile whose earlier
+    weights are already taken.  The inputs are checked to contain such rows."""
+    lay = _layout(dtype, H, Hkv, D, bs, lens, nq, seed=7)
+    ten = wl.make_prefill_tensors(lay, device="cuda")
+    rng = np.random.default_rng(11)
+    k = ten["k_cache"]
+    for s, L in enumerate(lay.context_lens):
+        for pos in rng.choice(np.arange(140, int(L)), size=8, replace=False):
+            k[int(lay.block_tables[s, pos // bs]), :, int(pos % bs), :] *= 8
+    # rows whose keys past the first tile reach 8 (log2 units) above that tile's maximum
+    qf, kf = ten["q"].float().cpu().numpy(), k.float().cpu().numpy()
+    qsl, nqs, G = lay.extra["query_start_loc"], lay.extra["query_lens"], H // Hkv
+    jumps = 0
+    for s, L in enumerate(lay.context_lens):
+        L, n = int(L), int(nqs[s])
+        keys = np.concatenate([kf[lay.block_tables[s, b]] for b in range((L + bs - 1) // bs)], axis=1)[:, :L]
+        for i in range(max(0, 128 - (L - n)), n):
+            pos = L - n + i
+            lg = np.einsum("hd,hkd->hk", qf[qsl[s] + i].reshape(Hkv, G, D).reshape(H, D),
+                           np.repeat(keys[:, :pos + 1], G, axis=0)) * lay.scale * np.log2(np.e)
+            jumps += int((lg[:, 128:].max(axis=1) > lg[:, :128].max(axis=1) + 8).sum())
+    assert jumps > 0
+    out, err = _gpu(lay, ten)
+    assert err == 0
+    # one key dominates such a row, so outputs reach |v| ~ 4, where the bf16
+    # spacing alone (2^-5 on [4, 8)) exceeds the absolute 1e-2: the bar grows
+    # with the output's magnitude (rounding of P and of the output, 2^-8
+    # relative each, with room for accumulation)
+    ref = _oracle(lay, ten)
+    got = oracle.decode(raw(out, dtype), dtype)
+    e = np.abs(got - ref)
+    stats = dict(max_abs=float(e.max()), mean_abs=float(e.mean()), max_ref=float(np.abs(ref).max()),
+                 worst_ratio=float((e / (1e-2 + 2.0 ** -6 * np.abs(ref))).max()))
+    print(stats)
+    assert np.isfinite(got).all()
+    assert (e <= 1e-2 + 2.0 ** -6 * np.abs(ref)).all(), stats
+    assert stats["mean_abs"] <= 1e-3, stats
+
+
 @pytest.mark.parametrize("name", sorted(wl.PREFILL_CONFIGS))
 def test_prefill_full_size_sampled(name):
     """The full workload in the launch the bench times; 48 sampled query rows
