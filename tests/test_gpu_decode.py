@@ -12,7 +12,7 @@ import torch
 import oracle
 import paged_kv_cache_480_b200 as pkv
 from paged_kv_cache_480_b200 import workloads as wl
-from gpu_helpers import check_step, compare, gpu_step, host_copy, oracle_step, raw, same_bits
+from gpu_helpers import check_step, compare, compare_scaled, gpu_step, host_copy, oracle_step, raw, same_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -22,6 +22,33 @@ def _lib():
     from paged_kv_cache_480_b200 import build
     build.build()
     pkv.load_library()
+
+
+# ---------------------------------------------------------------------------
+# keys whose logits jump far above the rest of the context
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,ps", [("llama7b_bf16", 0), ("gqa_long_bf16", 0), ("gqa_long_bf16", 512),
+                                     ("opt13b_f16", 0), ("tiny_mha_f32", 16)])
+def test_decode_logit_jumps(name, ps):
+    """Unit-variance inputs with the keys of random context positions scaled
+    by 8: single keys dominate their rows, wherever they fall in a slice,
+    block or partition (the merge sees partitions with very different
+    maxima)."""
+    lay = wl.make_layout(name, num_seqs=min(8, wl.make_layout(name).num_seqs))
+    lay.value_scale = 1.0
+    ten = wl.make_tensors(lay, device="cuda")
+    rng = np.random.default_rng(5)
+    bs = lay.block_size
+    for s, L in enumerate(lay.context_lens):
+        L = int(L)
+        if L < 2:
+            continue
+        for pos in rng.choice(np.arange(L - 1), size=min(6, L - 1), replace=False):   # not the new token
+            ten["k_cache"][int(lay.block_tables[s, pos // bs]), :, int(pos % bs), :] *= 8
+    host = host_copy(ten, lay.dtype)
+    out, err = gpu_step(lay, ten, ps)
+    assert err == 0
+    compare_scaled(out, oracle_step(lay, host), lay.dtype)
 
 
 # ---------------------------------------------------------------------------
