@@ -36,6 +36,18 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
 
 
+def test_python_names_cover_the_entry_points():
+    """Every public name of the package resolves, and every C entry point that
+    computes has a Python function of the same name."""
+    import paged_kv_cache_480_b200 as pkv
+    for n in pkv.__all__:
+        assert getattr(pkv, n) is not None, n
+    for n in declared_functions():
+        if n.startswith(("paged_attention", "reshape_and_cache", "copy_blocks", "swap_blocks")) \
+                and n != "paged_attention_workspace_init":
+            assert n in pkv.__all__, f"{n} has no Python name"
+
+
 def test_status_strings(lib):
     assert lib.pkv_status_string(0) == b"ok"
     assert b"sm_100a" in lib.pkv_version()
