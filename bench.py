@@ -177,8 +177,9 @@ def build_cow_state(device):
 # ---------------------------------------------------------------------------
 class ClockSampler:
     """SM clock and clock-event reasons of this process's GPU, polled through
-    NVML every 2 ms on a background thread while the timed region runs (it
-    only reads; no setting is changed).  Samples are kept only between
+    NVML every 0.25 ms on a background thread while the timed region runs
+    (it only reads; no setting is changed; a decode step is ~0.25 ms, so a
+    20-step region still gets ~20 samples).  Samples are kept only between
     mark_start() and mark_end(), i.e. under load."""
 
     REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
@@ -219,7 +220,7 @@ class ClockSampler:
                     mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                     bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
                     self.samples.append((float(mhz), [k for k, m in masks.items() if bits & m]))
-                self._stop.wait(0.002)
+                self._stop.wait(0.00025)
         except Exception as e:              # NVML missing: report no samples
             self.error = str(e)[:120]
 
@@ -246,7 +247,7 @@ class ClockSampler:
                     "source": "nvml", "error": self.error}
         reasons = sorted({r for _, rs in self.samples for r in rs})
         return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 2 ms polling"}
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 0.25 ms polling"}
 
 
 def kernel_source_sha():
