@@ -34,7 +34,9 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 200 on the GPU, so that the clock samples taken during the "
+                         "timed region are many even for a 0.25 ms step; 20 for the CPU reference arm)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="opt13b_f16")
@@ -51,7 +53,10 @@ def parse():
                     help="fp8: E4M3 cache written by reshape_and_cache_fp8kv, read by the fp8 decode")
     ap.add_argument("--fused", action="store_true",
                     help="cache write fused into the decode (paged_attention_decode_append)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 200
+    return args
 
 
 def peaks():
