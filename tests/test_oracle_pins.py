@@ -412,6 +412,29 @@ def test_prefill_matches_causal_sdpa(dtype, H, Hkv, D, bs, lens, nq):
             np.testing.assert_allclose(got[qsl[s]:qsl[s + 1]], ref2.transpose(0, 1).numpy(), atol=1e-12)
 
 
+def test_prefill_large_logits_match_causal_sdpa():
+    """Logits of tens (the scale 8x the usual): the oracle's exponentials stay
+    finite and it still equals causal SDPA in fp64, the definition the
+    logit-jump GPU tests rely on."""
+    rng = np.random.default_rng(32)
+    lens, nq = [300, 150], [300, 60]
+    H, Hkv, D, bs = 4, 2, 64, 16
+    _, Kc, Vc, kc, vc, _, tables = build_paged(rng, lens, H, Hkv, D, bs, "bf16")
+    qsl = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    qt = torch.from_numpy(rng.standard_normal((int(qsl[-1]), H, D))).to(torch.bfloat16)
+    scale = 8.0 / math.sqrt(D)
+    got = oracle.paged_prefill(_raw_from_torch(qt, "bf16"), kc, vc, tables, np.array(lens, np.int32), qsl,
+                               scale, "bf16", Hkv, bs)
+    assert np.isfinite(got).all()
+    G = H // Hkv
+    for s, (L, n) in enumerate(zip(lens, nq)):
+        K, V = Kc[s].repeat_interleave(G, 0), Vc[s].repeat_interleave(G, 0)
+        q = qt[qsl[s]:qsl[s + 1]].double().transpose(0, 1)
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(got[qsl[s]:qsl[s + 1]], ref.transpose(0, 1).numpy(), rtol=0, atol=1e-11)
+
+
 def test_prefill_last_query_equals_decode():
     """The last query of every sequence attends to the whole context: the decode definition."""
     rng = np.random.default_rng(31)
