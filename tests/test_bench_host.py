@@ -112,3 +112,24 @@ def test_prefill_flop_model():
     # the slot of sequence 1's last query is its last context position
     L, bs = 300, 16
     assert slots[5 + 16] == lay.block_tables[1, (L - 1) // bs] * bs + (L - 1) % bs
+
+
+def test_default_steps_depend_on_the_arm(monkeypatch):
+    """No --steps: 200 timed steps on the GPU arms (so that a 0.25 ms decode
+    step still leaves many clock samples inside the timed region), 20 for the
+    CPU reference arm; an explicit --steps is kept as given."""
+    cases = [([], 200), (["--impl", "reference"], 20), (["--measure", "prefill"], 200),
+             (["--steps", "7"], 7), (["--impl", "reference", "--steps", "3"], 3)]
+    for argv, steps in cases:
+        monkeypatch.setattr(sys, "argv", ["bench.py"] + argv)
+        assert bench.parse().steps == steps, argv
+
+
+def test_clock_summary_median_and_reasons():
+    clk = bench.ClockSampler(0)
+    clk.samples = [(1965.0, []), (1900.0, ["sw_power_cap"]), (1965.0, [])]
+    clk.max_mhz = 1965.0
+    s = clk.summary()
+    assert s["sm_mhz"] == 1965.0 and s["samples"] == 3 and s["reasons"] == ["sw_power_cap"]
+    empty = bench.ClockSampler(0).summary()
+    assert empty["samples"] == 0 and empty["sm_mhz"] is None
