@@ -4,8 +4,10 @@ One step = one pass of the whole hot path over one batch: copy-on-write block
 copies (when the workload forks), the cache write of each sequence's new
 token, and paged decode attention (plus its log-sum-exp merge when contexts
 are split).  Inputs are seeded and synthetic, resident in HBM when timing
-starts; the K/V of a step (1.5 GB for the default workload) is far larger
-than the 126 MB L2, so no explicit flush is needed.
+starts; the K/V of a step (4.3 GB for the default workload, the 7B-shaped
+layer of 256 sequences) is far larger than the 126 MB L2, so no explicit
+flush is needed.  The same line also reports, under "targets", the decode
+call of the long-context GQA and MQA workloads timed the same way.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the CPU oracle as the reference arm)
@@ -39,7 +41,7 @@ def parse():
                          "timed region are many even for a 0.25 ms step; 20 for the CPU reference arm)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="opt13b_f16")
+    ap.add_argument("--workload", default="llama7b_bf16")
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -53,6 +55,8 @@ def parse():
                     help="fp8: E4M3 cache written by reshape_and_cache_fp8kv, read by the fp8 decode")
     ap.add_argument("--fused", action="store_true",
                     help="cache write fused into the decode (paged_attention_decode_append)")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the decode calls of the long-context GQA / MQA workloads")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = 20 if args.impl == "reference" else 200
@@ -284,7 +288,7 @@ def profiled_prefill_traffic(workload):
     return e.get("bytes_per_call")
 
 
-def profiled_traffic(workload, block_size):
+def profiled_traffic(workload, block_size, fp8=False):
     """DRAM bytes per decode call from a committed ncu summary, if it still
     matches the kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
@@ -292,7 +296,7 @@ def profiled_traffic(workload, block_size):
         return None
     with open(path) as f:
         d = json.load(f)
-    key = f"{workload}/bs{block_size}"
+    key = f"{workload}/bs{block_size}" + ("/fp8" if fp8 else "")
     e = d.get(key)
     if not e or e.get("source_sha") != kernel_source_sha():
         return None
@@ -302,9 +306,10 @@ def profiled_traffic(workload, block_size):
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(lay, host, budget_s, max_seqs=None, threads=None):
+def oracle_sample(lay, host, budget_s, max_seqs=None, threads=None, fp8=False):
     """Time the oracle on leading sequences of the workload (bounded), repeating
-    until ~budget_s of work; returns (GB/s, seconds, bytes, seqs, threads)."""
+    until ~budget_s of work; returns (GB/s, seconds, bytes, seqs, threads).
+    fp8: the caches hold E4M3 codes (FP8_SCALES) and the oracle's FP8 decode runs."""
     import oracle
     S = lay.num_seqs if max_seqs is None else min(max_seqs, lay.num_seqs)
     sub = lambda a: a[:S]
@@ -312,13 +317,18 @@ def oracle_sample(lay, host, budget_s, max_seqs=None, threads=None):
     from paged_kv_cache_480_b200 import workloads as wl
     sublay = wl.Layout(**{**lay.__dict__, "num_seqs": S, "context_lens": sub(lay.context_lens),
                           "block_tables": sub(lay.block_tables), "slot_mapping": sub(lay.slot_mapping)})
-    nbytes = decode_bytes(sublay)
+    nbytes = decode_bytes(sublay, 1 if fp8 else None)
     total_t, total_b, reps = 0.0, 0, 0
     while total_t < budget_s or reps == 0:
         t0 = time.perf_counter()
-        oracle.paged_attention(host["q"][:S], host["k_cache"], host["v_cache"], sublay.block_tables,
-                               sublay.context_lens, lay.scale, lay.dtype, lay.num_kv_heads,
-                               lay.block_size, nthreads=threads)
+        if fp8:
+            oracle.paged_attention_fp8(host["q"][:S], lay.dtype, host["k_cache"], host["v_cache"], *FP8_SCALES,
+                                       sublay.block_tables, sublay.context_lens, lay.scale, lay.num_kv_heads,
+                                       lay.block_size, nthreads=threads)
+        else:
+            oracle.paged_attention(host["q"][:S], host["k_cache"], host["v_cache"], sublay.block_tables,
+                                   sublay.context_lens, lay.scale, lay.dtype, lay.num_kv_heads,
+                                   lay.block_size, nthreads=threads)
         total_t += time.perf_counter() - t0
         total_b += nbytes
         reps += 1
@@ -332,7 +342,10 @@ def host_arrays(ten, dtype):
     out = {}
     for k in ("q", "k_cache", "v_cache"):
         t = ten[k].contiguous().cpu()
-        out[k] = t.numpy() if dtype == "f32" else t.view(torch.int16).numpy().view(np.uint16)
+        if t.dtype == torch.uint8:                  # E4M3 codes
+            out[k] = t.numpy()
+        else:
+            out[k] = t.numpy() if dtype == "f32" else t.view(torch.int16).numpy().view(np.uint16)
     return out
 
 
@@ -491,7 +504,7 @@ def run_ours(args, rank, world, local_rank):
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind,
                 "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
-                "traffic": None if fp8 else profiled_traffic(lay.name, bs),
+                "traffic": profiled_traffic(lay.name, bs, fp8),
                 "algorithmic_bytes": decode_bytes(lay, cb),
                 "avg_call_us": dec_avg * 1e3}
         result = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -512,23 +525,106 @@ def run_ours(args, rank, world, local_rank):
                              "parallelism": f"replicas x{world}"},
                   "roofline": roof, "gpu_launches": launches_per_step * args.steps,
                   "clocks": clk.summary(), "device_errors": errors}
-        if not args.no_e2e and not fp8:
-            result["e2e"] = run_e2e(args, lay, ten, pairs, device, ws, step_bytes)
-        if not args.no_cpu_baseline and world == 1 and not fp8:
+        if not args.no_e2e:
+            result["e2e"] = run_e2e(args, lay, ten, pairs, device, ws, step_bytes, fp8)
+        if not args.no_cpu_baseline and world == 1:
             host = host_arrays(ten, lay.dtype)
+            what = "fp64 oracle (FP8 decode)" if fp8 else "fp64 oracle"
             gbs, t, b, seqs, threads = oracle_sample(lay, host, 10.0,
-                                                     max_seqs=max(1, lay.num_seqs // 8))
-            gbs1, t1, _, seqs1, _ = oracle_sample(lay, host, 5.0, max_seqs=max(1, lay.num_seqs // 32), threads=1)
+                                                     max_seqs=max(1, lay.num_seqs // 8), fp8=fp8)
+            gbs1, t1, _, seqs1, _ = oracle_sample(lay, host, 5.0, max_seqs=max(1, lay.num_seqs // 32),
+                                                  threads=1, fp8=fp8)
             result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                      "sample": f"fp64 oracle over the first {max(1, lay.num_seqs // 8)} "
+                                      "sample": f"{what} over the first {max(1, lay.num_seqs // 8)} "
                                                 f"sequences, repeated: {seqs} sequence-passes in {t:.1f} s",
                                       "value_1core": gbs1,
                                       "sample_1core": f"first {max(1, lay.num_seqs // 32)} sequences on one "
                                                       f"thread: {seqs1} sequence-passes in {t1:.1f} s"}
+        if not args.no_targets and not args.fused:
+            del ten, out, ws
+            torch.cuda.empty_cache()
+            result["targets"] = decode_targets(args, device, local_rank, fp8,
+                                               exclude=lay.name if args.partition_size == 0 else None)
     return result
 
 
-def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
+TARGET_WORKLOADS = ("gqa_long_bf16", "mqa_long_bf16")
+
+
+def decode_targets(args, device, local_rank, fp8, exclude=None):
+    """The decode call of the long-context workloads (GQA: 64 query heads
+    over 8 KV heads; MQA: 64 over 1; 16 sequences of 16K-32K tokens), each
+    timed like the main line's: one reshape_and_cache + decode per step, CUDA
+    events around the decode call on its stream, args.steps calls after
+    args.warmup, SM clocks sampled meanwhile."""
+    import torch
+    import paged_kv_cache_480_b200 as pkv
+    from paged_kv_cache_480_b200 import workloads as wl
+    peak, peak_kind = peaks()
+    cb = 1 if fp8 else None
+    res = {}
+    for name in TARGET_WORKLOADS:
+        if name == exclude:
+            continue
+        lay, ten, _ = build_workload(name, None, device, fp8)
+        S, H, Hkv, D, bs = lay.num_seqs, lay.num_heads, lay.num_kv_heads, lay.head_size, lay.block_size
+        max_ctx = lay.max_context_len
+        bt = torch.from_numpy(lay.block_tables).to(device)
+        cl = torch.from_numpy(lay.context_lens).to(device)
+        sm = torch.from_numpy(lay.slot_mapping).to(device)
+        out = torch.empty_like(ten["q"])
+        need = pkv.paged_attention_workspace_size(S, H, Hkv, D, bs, max_ctx, {"f32": 0, "f16": 1, "bf16": 2}[lay.dtype])
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        stream = torch.cuda.current_stream(device)
+        ev = []
+
+        def step(record=False):
+            if fp8:
+                pkv.reshape_and_cache_fp8kv(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm,
+                                            *FP8_SCALES, stream=stream)
+            else:
+                pkv.reshape_and_cache(ten["k_new"], ten["v_new"], ten["k_cache"], ten["v_cache"], sm, stream=stream)
+            if record:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            if fp8:
+                pkv.paged_attention_decode_fp8kv(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                                                 *FP8_SCALES, max_context_len=max_ctx, workspace=ws, stream=stream)
+            else:
+                pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                                           max_context_len=max_ctx, workspace=ws, stream=stream)
+            if record:
+                b.record(stream)
+                ev.append((a, b))
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize(device)
+        with ClockSampler(local_rank) as clk:
+            time.sleep(0.05)
+            clk.mark_start()
+            for _ in range(args.steps):
+                step(record=True)
+            torch.cuda.synchronize(device)
+            clk.mark_end()
+        errors = pkv.read_device_errors()
+        dec = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+        nbytes = decode_bytes(lay, cb)
+        gbs = nbytes / (dec * 1e-3) / 1e9
+        res[name] = {"avg_call_us": dec * 1e3, "achieved": gbs, "unit": "GB/s", "peak": peak, "peak_kind": peak_kind,
+                     "frac": gbs / peak, "frac_of_nominal_8TBs": gbs / NOMINAL_HBM_GBS,
+                     "algorithmic_bytes": nbytes, "seqs_per_s": S / (dec * 1e-3),
+                     "shape": f"{S} seqs, {H} q heads / {Hkv} KV heads, D {D}, bs {bs}, "
+                              f"mean context {float(lay.context_lens.mean()):.0f}",
+                     "kv_cache": "fp8-e4m3" if fp8 else lay.dtype, "calls": len(ev),
+                     "clocks": clk.summary(), "device_errors": errors}
+        del ten, out, ws
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_e2e(args, lay, ten, pairs, device, ws, step_bytes, fp8=False):
     """Same step through the C ABI with the step's inputs in pinned host
     memory.  The inputs (q, new K/V, slots, tables, lengths, CoW pairs) sit
     in one pinned staging buffer and go to the device in one copy; the
@@ -567,7 +663,13 @@ def run_e2e(args, lay, ten, pairs, device, ws, step_bytes):
         d_buf.copy_(h_buf, non_blocking=True)
         if "pairs" in d:
             pkv.copy_blocks([ten["k_cache"]], [ten["v_cache"]], d["pairs"], stream=stream)
-        if args.fused:
+        if fp8:
+            pkv.reshape_and_cache_fp8kv(d["k"], d["v"], ten["k_cache"], ten["v_cache"], d["sm"], *FP8_SCALES,
+                                        stream=stream)
+            pkv.paged_attention_decode_fp8kv(out, d["q"], ten["k_cache"], ten["v_cache"], d["bt"], d["cl"],
+                                             lay.scale, *FP8_SCALES, max_context_len=max_ctx, workspace=ws,
+                                             stream=stream)
+        elif args.fused:
             pkv.paged_attention_decode_append(out, d["q"], d["k"], d["v"], ten["k_cache"], ten["v_cache"],
                                               d["sm"], d["bt"], d["cl"], lay.scale,
                                               max_context_len=max_ctx, workspace=ws, stream=stream)

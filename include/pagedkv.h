@@ -32,7 +32,8 @@
  *            block manager owns host memory only (create/destroy).
  *   Streams  GPU calls are asynchronous on the given cudaStream_t (passed as
  *            void*, NULL = the legacy default stream); they never
- *            synchronise, except pkv_read_device_errors.
+ *            synchronise, except pkv_read_device_errors.  The stream must
+ *            belong to the current device (PKV_ERR_INVALID_ARG otherwise).
  *   Errors   argument errors are found on the host before anything is
  *            launched and return a status with nothing launched.  A failed
  *            launch returns PKV_ERR_CUDA.  Conditions only the device can see
@@ -72,6 +73,7 @@ typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
 #define PKV_DEVERR_CONTEXT 4u   /* context_len < 0, > max_blocks_per_seq * block_size or > max_context_len */
 #define PKV_DEVERR_COPY_ID 8u   /* a copy_blocks pair outside [0, num_blocks) */
 #define PKV_DEVERR_WAIT 16u     /* a bounded wait for an asynchronous copy gave up */
+#define PKV_DEVERR_COPY_OVERLAP 32u /* copy pairs whose result would depend on their order */
 
 const char* pkv_status_string(pkv_status status);
 const char* pkv_version(void);
@@ -96,7 +98,7 @@ const char* pkv_version(void);
  *                  step's own token once reshape_and_cache wrote it)
  *   scale          softmax scale (usually 1/sqrt(head_size))
  *   num_kv_heads   KV heads; num_heads must be a multiple (G = num_heads /
- *                  num_kv_heads in {1, 2, 4, 8})
+ *                  num_kv_heads, any value: MHA, GQA and MQA)
  *   block_size     tokens per block, 16 or 32
  *   num_seqs ... max_blocks_per_seq   the sizes above
  *   max_context_len host-known upper bound of context_lens (> 0); sizes the
@@ -112,12 +114,15 @@ const char* pkv_version(void);
  *                  paged_attention_workspace_size(...) bytes.  Its first 256
  *                  bytes hold scheduling counters that must be zero before
  *                  the first use (paged_attention_workspace_init, or a
- *                  zero-filled allocation); every call leaves them zero.
+ *                  zero-filled allocation); every call leaves them zero,
+ *                  also one whose bounded waits gave up (PKV_DEVERR_WAIT).
  *                  Calls that run concurrently need separate workspaces.
  *   stream         cudaStream_t (void*), may be NULL
  *
  * Supported: dtype f32/f16/bf16, head_size 64 or 128, block_size 16 or 32,
- * G in {1, 2, 4, 8}, num_seqs <= 16384.  Anything else: PKV_ERR_UNSUPPORTED.
+ * any G, num_seqs <= 16384.  Anything else: PKV_ERR_UNSUPPORTED.  Groups of
+ * more than 8 query heads are processed in slices of 8 heads that stream the
+ * same K/V tiles at about the same time (the repeats come from L2).
  * ------------------------------------------------------------------------- */
 pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                                   const void* v_cache, const int32_t* block_tables,
@@ -170,9 +175,9 @@ pkv_status paged_attention_decode_append(void* out, const void* q, const void* k
  *   out[s, h, :] = sum_t softmax_t(scale * q . (k_scale * K_s[t])) v_scale * V_s[t],
  * q and out in `dtype` (f32, f16 or bf16).  Workspace, partitioning, checks
  * and errors as for paged_attention_decode (the workspace size does not
- * depend on the cache type).  With 16-bit q and 4 or 8 query heads per KV
- * head the products run on the tensor cores in fp16 (E4M3 is exact in fp16;
- * bf16 q is rounded to fp16 there, so |q| must stay below 65504).
+ * depend on the cache type).  With 16-bit q the products run on the tensor
+ * cores in fp16 (E4M3 is exact in fp16; bf16 q is rounded to fp16 there, so
+ * |q| must stay below 65504).
  *
  * reshape_and_cache_fp8kv: reshape_and_cache into such caches: each element
  * x of key (value) becomes e4m3(x / k_scale) (resp. v_scale), the quotient
@@ -242,8 +247,14 @@ pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, 
  * k_caches[l] and v_caches[l] becomes a copy of block block_mapping[i][0]
  * (summary page of the SOSP 2023 paper, sections 1 and 2: copy-on-write
  * when parallel samples or shared prefixes diverge).  A bit copy of
- * block_bytes bytes per block.  Destinations must be distinct and no
- * destination may also be a source (pairs are copied in parallel).
+ * block_bytes bytes per block.  Pairs are copied in parallel, so the result
+ * is that of copying them in any order only if destinations are distinct and
+ * no destination is also a source: a pair that shares its destination with
+ * another pair, or whose destination or source is another pair's source or
+ * destination, is skipped and sets PKV_DEVERR_COPY_OVERLAP (the other pairs
+ * are copied).  Several pairs may share one source (one shared block copied
+ * for several writers).  Each CTA checks its pair against the whole mapping,
+ * which adds num_pairs * 16 bytes of (cached) reads per block copied.
  *
  *   k_caches, v_caches HOST arrays of num_layers device pointers
  *   block_mapping  device, int64 [num_pairs][2] = (src, dst)
@@ -309,16 +320,14 @@ pkv_status paged_attention_decode_noalloc(void* out, const void* q, const void* 
  *   block_mapping  int64 [num_pairs][2] (src, dst) in device or pinned host
  *                  memory; ids outside [0, src_num_blocks) / [0,
  *                  dst_num_blocks) are skipped and flag PKV_DEVERR_COPY_ID
- * Destinations must be distinct.  Asynchronous on the stream; the host pool
+ * Destinations must be distinct: pairs that share a destination are skipped
+ * and set PKV_DEVERR_COPY_OVERLAP.  Asynchronous on the stream; the host pool
  * must stay alive until the stream has passed the copy.
  * ------------------------------------------------------------------------- */
 pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, int num_caches,
                        const int64_t* block_mapping, int num_pairs, int src_num_blocks,
                        int dst_num_blocks, int64_t block_bytes, void* stream);
 
-/* Synchronise the stream, return the sticky device-check bits of the
- * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
- * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */
 /* ---------------------------------------------------------------------------
  * paged_attention_prefill -- causal attention of a batch of prompts, or of
  * prompt chunks, whose keys and values are already in the paged cache.
@@ -355,8 +364,10 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
  * block_size or queries outside [0, num_tokens) set PKV_DEVERR_CONTEXT and
  * the sequence's rows are not written; a block id outside the pool sets
  * PKV_DEVERR_BLOCK_ID and reads as zeros.
- * Supported: head_size 64 or 128, block_size 16 or 32, G in {1, 2, 4, 8},
- * num_blocks * num_kv_heads * block_size < 2^31.  f32: PKV_ERR_UNSUPPORTED.
+ * Supported: head_size 64 or 128, block_size 16 or 32, G = num_heads /
+ * num_kv_heads from 1 to 128 (a query tile of 128 rows holds floor(128 / G)
+ * queries of G heads), num_blocks * num_kv_heads * block_size < 2^31.
+ * f32: PKV_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------- */
 pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache,
                                    const void* v_cache, const int32_t* block_tables,
@@ -366,7 +377,21 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
                                    int num_blocks, int max_blocks_per_seq, int max_query_len,
                                    pkv_dtype dtype, void* stream);
 
+/* Synchronise the stream, return the sticky device-check bits of the
+ * current device in *bits and clear them.  Returns PKV_ERR_DEVICE_CHECK if
+ * any bit was set, else PKV_OK (or PKV_ERR_CUDA). */
 pkv_status pkv_read_device_errors(void* stream, uint32_t* bits);
+
+/* For tests of the failure path: every wait of the decode and prefill kernels
+ * for an asynchronous copy, a tensor-core commit or another warp's result
+ * gives up after `polls` polls (each may suspend the thread for a short
+ * hardware-defined time), skips the rest of its work, lets the copies it
+ * already issued land, frees what it holds and sets PKV_DEVERR_WAIT; the
+ * outputs of that call are then undefined.  polls = 0 gives up at the first
+ * wait; polls < 0 restores the default (2^22, far beyond any real latency).
+ * Process-wide; applies to calls launched after it returns.  polls above
+ * 2^32 - 1: PKV_ERR_INVALID_ARG. */
+pkv_status pkv_set_wait_limit(int64_t polls);
 
 /* ---------------------------------------------------------------------------
  * Host block manager (KV-cache manager of the summary page, section 2; the

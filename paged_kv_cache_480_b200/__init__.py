@@ -16,7 +16,8 @@ __all__ = [
     "paged_attention_decode", "paged_attention_decode_append", "paged_attention_decode_fp8kv",
     "paged_attention_decode_noalloc", "paged_attention_prefill",
     "reshape_and_cache_fp8kv", "paged_attention_workspace_size", "paged_attention_partition_size",
-    "reshape_and_cache", "copy_blocks", "swap_blocks", "read_device_errors", "BlockManager", "load_library",
+    "reshape_and_cache", "copy_blocks", "swap_blocks", "read_device_errors", "set_wait_limit", "BlockManager",
+    "load_library",
     "PagedKVError", "OutOfBlocks", "default_workspace",
 ]
 

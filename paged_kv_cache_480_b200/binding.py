@@ -17,7 +17,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CU
           4: "out of blocks", 5: "unknown or duplicate sequence id", 6: "workspace too small",
           7: "a device-side check fired"}
 DEVERR = {1: "block id out of range", 2: "slot out of range", 4: "context length out of range",
-          8: "copy pair out of range", 16: "bounded wait gave up"}
+          8: "copy pair out of range", 16: "bounded wait gave up", 32: "copy pairs overlap"}
 
 
 class PagedKVError(RuntimeError):
@@ -78,6 +78,8 @@ def load_library(path=LIB_PATH):
         lib.paged_attention_prefill.restype = I
         lib.pkv_read_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         lib.pkv_read_device_errors.restype = I
+        lib.pkv_set_wait_limit.argtypes = [I64]
+        lib.pkv_set_wait_limit.restype = I
         lib.pkv_bm_create.argtypes = [I, I, P, ctypes.POINTER(P)]
         lib.pkv_bm_create.restype = I
         lib.pkv_bm_destroy.argtypes = [P]
@@ -457,6 +459,13 @@ def read_device_errors(stream=None):
     if st not in (0, 7):
         _check(st, "pkv_read_device_errors")
     return bits.value
+
+
+def set_wait_limit(polls):
+    """For tests of the failure path: polls after which the kernels' bounded
+    waits give up (pkv_set_wait_limit in pagedkv.h); negative restores the
+    default."""
+    _check(load_library().pkv_set_wait_limit(int(polls)), "pkv_set_wait_limit")
 
 
 class BlockManager:

@@ -44,6 +44,22 @@ __global__ void reshape_and_cache_kernel(const CacheWriteParams p) {
     }
 }
 
+// Pairs are copied in parallel, so a pair whose destination is also another
+// pair's destination or (within one pool) another pair's source, or whose
+// source is another pair's destination, would make the result depend on the
+// order the copies happen to run in.  Every CTA of a pair scans the whole
+// mapping (all threads of the CTA take part); such a pair is skipped.
+__device__ __forceinline__ bool pair_conflicts(const int64_t* map, int num_pairs, int pair, int64_t src,
+                                               int64_t dst, bool same_pool) {
+    bool hit = false;
+    for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+        if (j == pair) continue;
+        const int64_t sj = map[2 * (int64_t)j], dj = map[2 * (int64_t)j + 1];
+        hit |= dj == dst || (same_pool && (sj == dst || dj == src));
+    }
+    return __syncthreads_or(hit) != 0;
+}
+
 // grid = (pairs, layers, 2 caches); each CTA copies one block with 16-byte
 // vectors, four loads in flight per thread.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyBlocksParams p) {
@@ -54,6 +70,10 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyBlocksParams
     const int64_t dst = p.block_mapping[2 * (int64_t)pair + 1];
     if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
         if (threadIdx.x == 0 && layer == 0 && which == 0) flag_error(p.errors, PKV_DEVERR_COPY_ID);
+        return;
+    }
+    if (pair_conflicts(p.block_mapping, p.num_pairs, pair, src, dst, true)) {
+        if (threadIdx.x == 0 && layer == 0 && which == 0) flag_error(p.errors, PKV_DEVERR_COPY_OVERLAP);
         return;
     }
     unsigned char* base = static_cast<unsigned char*>(which ? p.v[layer] : p.k[layer]);
@@ -85,6 +105,10 @@ __global__ void __launch_bounds__(256) swap_blocks_kernel(const SwapBlocksParams
     const int64_t dst = p.block_mapping[2 * (int64_t)pair + 1];
     if (src < 0 || src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
         if (threadIdx.x == 0 && c == 0) flag_error(p.errors, PKV_DEVERR_COPY_ID);
+        return;
+    }
+    if (pair_conflicts(p.block_mapping, p.num_pairs, pair, src, dst, false)) {
+        if (threadIdx.x == 0 && c == 0) flag_error(p.errors, PKV_DEVERR_COPY_OVERLAP);
         return;
     }
     const uint4* s = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(p.src[c]) +

@@ -28,6 +28,7 @@ struct CopyBlocksParams {
     unsigned int* errors;
     int64_t block_bytes;
     int64_t num_blocks;
+    int num_pairs;
 };
 
 struct SwapBlocksParams {
@@ -37,6 +38,7 @@ struct SwapBlocksParams {
     unsigned int* errors;
     int64_t block_bytes;
     int64_t src_blocks, dst_blocks;
+    int num_pairs;
 };
 
 struct CacheWriteFp8Params {

@@ -5,9 +5,14 @@
 // block through the block table).
 //
 // Work decomposition
-//   item   = (sequence s, KV head g, partition p): tokens
-//            [p * PS, min(L_s, (p + 1) * PS)) of one KV head, for all G query
-//            heads of the group (each K/V byte is read from HBM once).
+//   item   = (sequence s, KV head g, partition p, head slice): tokens
+//            [p * PS, min(L_s, (p + 1) * PS)) of one KV head, for the query
+//            heads of the group (each K/V byte is read from HBM once).  A
+//            group of up to 8 query heads is one slice, padded to the kernel's
+//            column count GP in {1, 2, 4, 8}; a larger group is split into
+//            slices of 8 heads whose items follow each other, so their warps
+//            stream the same tiles at about the same time and all but the
+//            first read them from L2.
 //   warp   = one item at a time.  A warp streams its item's (block, head)
 //            K and V tiles -- bs x head_size contiguous bytes each -- into a
 //            private ring of R shared-memory stages with untiled bulk copies
@@ -59,32 +64,40 @@ struct DecodeParams {
     const void* value;
     const int64_t* slot_mapping;
     int64_t key_stride, value_stride;   // elements between sequences
+    int group;              // G = num_heads / num_kv_heads (any value >= 1)
+    int slices;             // head slices per group: ceil(G / GP)
+    uint32_t wait_limit;    // polls before a wait for a stage's copies gives up
     int stages;             // R
     int warps;              // W consumer warps per CTA
     uint32_t warp_smem;     // bytes of one warp's region
     uint32_t seq_smem;      // bytes of the per-CTA length / prefix arrays
 };
 
-// TQ: element type of q and out; TC: element type of the caches.
+// TQ: element type of q and out; TC: element type of the caches; G: query-head
+// columns of one item (the group size padded to 1, 2, 4 or 8).
 template <typename TQ, typename TC, int D, int BS, int G>
 struct DecodeShape {
     static constexpr int EPC = Elem<TC>::kPerChunk;  // cache elements per 16-byte chunk
     static constexpr int ROW = D * (int)sizeof(TC);  // bytes per cache token row
     static constexpr int TILE = BS * ROW;            // bytes per (block, KV head) tile
     static constexpr int QROW = D * (int)sizeof(TQ); // bytes per q / out row
-    static constexpr int QBYTES = G * QROW;          // q rows of one group
+    static constexpr int QBYTES = G * QROW;          // q rows of one item, at most
 };
 
 struct StageMeta {
-    int item, s, g, part;
-    int nvalid;  // valid tokens in this block (0 = nothing to read)
-    int flags;   // kFirst | kLast | kWhole
+    int64_t pidx;   // first partial row of the item: partition index * num_heads + first head
+    int64_t obase;  // first output row: s * num_heads + first head
+    int64_t slot;   // fused cache write: the new token's slot
+    int g;          // KV head
+    int nh;         // query heads of the item (<= GP)
+    int nvalid;     // valid tokens in this block (0 = nothing to read)
+    int flags;      // kFirst | kLast | kWhole | kStore
     int qslot;
-    int newrow;  // row of this block that takes the step's new token, or -1
-    int64_t slot;
-    int64_t pad;
+    int newrow;     // row of this block that takes the step's new token, or -1
 };
-constexpr int kFirst = 1, kLast = 2, kWhole = 4;
+// kStore: this item also stores the step's new token into the cache (one
+// head slice of a group does)
+constexpr int kFirst = 1, kLast = 2, kWhole = 4, kStore = 8;
 
 // Host and device agree on this layout of one warp's shared-memory region.
 template <typename TQ, typename TC, int D, int BS, int G>
@@ -109,7 +122,9 @@ struct WarpSmem {
 
 struct Item {
     int idx;      // item index (>= n_items: none)
-    int s, g, part;
+    int s;
+    int vg;       // KV head * slices + head slice
+    int jsp;      // partition index over the batch (partitions of sequences before s, plus this one's)
     int tok0;     // first token
     int ntok;     // tokens in the item (may be 0 for an empty sequence)
     int nblk;     // stages the item occupies (>= 1)
@@ -165,14 +180,20 @@ struct FmaConsumer {
         for (int d = 0; d < DL; ++d) qf[d] = acc[d] = 0.f;
     }
 
-    __device__ __forceinline__ void begin(const unsigned char* qslot, float qscale) {
+    // nh: heads of the item; lanes of the padding heads hold q = 0 and write nothing
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float qscale, int nh) {
         const uint4* qrow = reinterpret_cast<const uint4*>(qslot + h * S::QROW);
 #pragma unroll
         for (int k = 0; k < CPL; ++k)
 #pragma unroll
             for (int j = 0; j < QPC; ++j) {
                 float f[EPQ];
-                Elem<TQ>::widen(qrow[(c + Q * k) * QPC + j], f);
+                if (h < nh) {
+                    Elem<TQ>::widen(qrow[(c + Q * k) * QPC + j], f);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPQ; ++e) f[e] = 0.f;
+                }
 #pragma unroll
                 for (int e = 0; e < EPQ; ++e) qf[k * EPC + j * EPQ + e] = f[e] * qscale;
             }
@@ -242,11 +263,10 @@ struct FmaConsumer {
 #pragma unroll
             for (int d = 0; d < DL; ++d) acc[d] += __shfl_xor_sync(kFull, acc[d], off);
         }
-        if (u != 0) return;
+        if (u != 0 || h >= mt.nh) return;
         if (mt.flags & kWhole) {
             const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
-            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<TQ*>(p.out) +
-                                                   ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + h) * D);
+            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<TQ*>(p.out) + (size_t)(mt.obase + h) * D);
 #pragma unroll
             for (int k = 0; k < CPL; ++k)
 #pragma unroll
@@ -258,7 +278,7 @@ struct FmaConsumer {
                 }
         } else {
             const float vs = p.v_scale;
-            float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + h) * D);
+            float4* prow = reinterpret_cast<float4*>(p.part_acc + (size_t)(mt.pidx + h) * D);
 #pragma unroll
             for (int k = 0; k < CPL; ++k)
 #pragma unroll
@@ -266,7 +286,7 @@ struct FmaConsumer {
                     prow[((c + Q * k) * EPC + e) / 4] =
                         make_float4(acc[k * EPC + e] * vs, acc[k * EPC + e + 1] * vs,
                                     acc[k * EPC + e + 2] * vs, acc[k * EPC + e + 3] * vs);
-            if (c == 0) p.part_ml[(size_t)mt.item * G + h] = make_float2(m_run, lt);
+            if (c == 0) p.part_ml[mt.pidx + h] = make_float2(m_run, lt);
         }
     }
 };
@@ -347,12 +367,12 @@ struct MmaConsumer {
         for (int j = 0; j < KJ; ++j) qf[j][0] = qf[j][1] = qf[j][2] = qf[j][3] = 0u;
     }
 
-    __device__ __forceinline__ void begin(const unsigned char* qslot, float) {
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float, int nh) {
         // B operand: column n = head r; rows = permuted dims of chunk 4j + c.
 #pragma unroll
         for (int j = 0; j < KJ; ++j) {
             uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (r < G) w = reinterpret_cast<const uint4*>(qslot + r * S::ROW)[4 * j + c];
+            if (r < nh) w = reinterpret_cast<const uint4*>(qslot + r * S::ROW)[4 * j + c];
             qf[j][0] = w.x;
             qf[j][1] = w.y;
             qf[j][2] = w.z;
@@ -458,30 +478,29 @@ struct MmaConsumer {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int head = 2 * c + e;
-            if (head >= G) continue;
+            if (head >= mt.nh) continue;
             const float lt = e ? t1 : t0;
             if (mt.flags & kWhole) {
                 const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
                 uint32_t words[MT];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) words[m] = Elem<T>::pack2(o[m][e] * inv, o[m][2 + e] * inv);
-                uint4* orow = reinterpret_cast<uint4*>(
-                    reinterpret_cast<T*>(p.out) +
-                    ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + head) * D + r * (D / 8));
+                uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) +
+                                                       (size_t)(mt.obase + head) * D + r * (D / 8));
 #pragma unroll
                 for (int ch = 0; ch < VCH; ++ch)
                     orow[ch] = make_uint4(words[4 * ch], words[4 * ch + 1], words[4 * ch + 2],
                                           words[4 * ch + 3]);
             } else {
                 const float vs = p.v_scale;
-                float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + head) * D +
+                float4* prow = reinterpret_cast<float4*>(p.part_acc + (size_t)(mt.pidx + head) * D +
                                                          r * (D / 8));
 #pragma unroll
                 for (int m = 0; m < MT; m += 2)
                     prow[m / 2] = make_float4(o[m][e] * vs, o[m][2 + e] * vs, o[m + 1][e] * vs,
                                               o[m + 1][2 + e] * vs);
                 if (r == 0)
-                    p.part_ml[(size_t)mt.item * G + head] = make_float2(e ? m1 : m0, lt);
+                    p.part_ml[mt.pidx + head] = make_float2(e ? m1 : m0, lt);
             }
         }
     }
@@ -556,11 +575,11 @@ struct MmaConsumerFp8 {
             for (int i = 0; i < 8; ++i) qf[j][i] = 0u;
     }
 
-    __device__ __forceinline__ void begin(const unsigned char* qslot, float) {
+    __device__ __forceinline__ void begin(const unsigned char* qslot, float, int nh) {
 #pragma unroll
         for (int j = 0; j < KJ; ++j) {
             uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-            if (r < G) {
+            if (r < nh) {
                 const uint4* qrow = reinterpret_cast<const uint4*>(qslot + r * S::QROW);
                 a = qrow[2 * (4 * j + c)];          // dims 16(4j+c) + 0..7
                 b = qrow[2 * (4 * j + c) + 1];      // dims 16(4j+c) + 8..15
@@ -745,30 +764,29 @@ struct MmaConsumerFp8 {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int head = 2 * c + e;
-            if (head >= G) continue;
+            if (head >= mt.nh) continue;
             const float lt = e ? t1 : t0;
             if (mt.flags & kWhole) {
                 const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
                 uint32_t words[MT];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) words[m] = Elem<TQ>::pack2(o[m][e] * inv, o[m][2 + e] * inv);
-                uint4* orow = reinterpret_cast<uint4*>(
-                    reinterpret_cast<TQ*>(p.out) +
-                    ((size_t)mt.s * p.num_heads + (size_t)mt.g * G + head) * D + r * (D / 8));
+                uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<TQ*>(p.out) +
+                                                       (size_t)(mt.obase + head) * D + r * (D / 8));
 #pragma unroll
                 for (int ch = 0; ch < MT / 4; ++ch)
                     orow[ch] = make_uint4(words[4 * ch], words[4 * ch + 1], words[4 * ch + 2],
                                           words[4 * ch + 3]);
             } else {
                 const float vs = p.v_scale;
-                float4* prow = reinterpret_cast<float4*>(p.part_acc + ((size_t)mt.item * G + head) * D +
+                float4* prow = reinterpret_cast<float4*>(p.part_acc + (size_t)(mt.pidx + head) * D +
                                                          r * (D / 8));
 #pragma unroll
                 for (int m = 0; m < MT; m += 2)
                     prow[m / 2] = make_float4(o[m][e] * vs, o[m][2 + e] * vs, o[m + 1][e] * vs,
                                               o[m + 1][2 + e] * vs);
                 if (r == 0)
-                    p.part_ml[(size_t)mt.item * G + head] = make_float2(e ? m1 : m0, lt);
+                    p.part_ml[mt.pidx + head] = make_float2(e ? m1 : m0, lt);
             }
         }
     }
@@ -822,7 +840,7 @@ __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, cons
         float fill[kMaxPartitionCandidates];
         float best = 0.f;
         for (int j = 0; j < nc; ++j) {
-            const float x = (float)s_count[j] * p.num_kv_heads / nw;
+            const float x = (float)s_count[j] * p.num_kv_heads * p.slices / nw;
             fill[j] = x / ceilf(x);
             best = fmaxf(best, fill[j]);
         }
@@ -905,28 +923,31 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
     griddep_launch();    // the merge kernel may get resident; it waits for our completion
 
     const int Hkv = p.num_kv_heads;
-    const int n_items = s_pre[nseq] * Hkv;
+    const int Gr = p.group;                      // real group size
+    const int NSL = p.slices;
+    const int NV = Hkv * NSL;                    // (KV head, slice) pairs per partition
+    const int n_items = s_pre[nseq] * NV;
     const int NW = gridDim.x * p.warps;
     const int gw = blockIdx.x * p.warps + warp;
 
     auto fetch = [&](int idx) -> Item {
         Item it;
         it.idx = idx;
-        it.s = it.g = it.part = it.tok0 = it.ntok = it.whole = it.tbl = 0;
+        it.s = it.vg = it.jsp = it.tok0 = it.ntok = it.whole = it.tbl = 0;
         it.nblk = 0;
         it.slot = -1;
         if (idx >= n_items) return it;
-        const int jsp = idx / Hkv;
-        it.g = idx - jsp * Hkv;
+        const int jsp = idx / NV;
+        it.vg = idx - jsp * NV;
+        it.jsp = jsp;
         int lo = 0, hi = nseq - 1;  // largest s with s_pre[s] <= jsp
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (s_pre[mid] <= jsp) lo = mid; else hi = mid - 1;
         }
         it.s = lo;
-        it.part = jsp - s_pre[lo];
         it.whole = (s_pre[lo + 1] - s_pre[lo]) == 1;
-        it.tok0 = it.part * PS;
+        it.tok0 = (jsp - s_pre[lo]) * PS;
         it.ntok = min(s_len[lo] - it.tok0, PS);
         const int used = (it.ntok + BS - 1) / BS;
         it.nblk = max(used, 1);
@@ -972,31 +993,39 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
             if (P.slot != (int64_t)phys * BS + newrow) newrow = -2;   // not the last position
         }
         if (lane == 0) {
+            int g = P.vg, sl = 0;                    // KV head and head slice
+            if (NSL > 1) {
+                g = P.vg / NSL;
+                sl = P.vg - g * NSL;
+            }
+            const int head0 = g * Gr + sl * G;       // first query head of the item
             StageMeta m;
-            m.item = P.idx; m.s = P.s; m.g = P.g; m.part = P.part;
+            m.pidx = (int64_t)P.jsp * p.num_heads + head0;
+            m.obase = (int64_t)P.s * p.num_heads + head0;
+            m.slot = P.slot;
+            m.g = g;
+            m.nh = min(G, Gr - sl * G);
             m.nvalid = nvalid;
-            m.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (P.whole ? kWhole : 0);
+            m.flags = (first ? kFirst : 0) | (last ? kLast : 0) | (P.whole ? kWhole : 0) | (sl == 0 ? kStore : 0);
             m.qslot = qslot_ctr;
             m.newrow = newrow < 0 ? -1 : newrow;
-            m.slot = P.slot;
-            m.pad = 0;
             meta[st] = m;
             const uint32_t bar = bar0 + 8 * st;
-            const uint32_t bytes = (first ? S::QBYTES : 0) + (nvalid > 0 ? 2 * S::TILE : 0) +
+            const uint32_t qbytes = (uint32_t)m.nh * S::QROW;
+            const uint32_t bytes = (first ? qbytes : 0) + (nvalid > 0 ? 2 * S::TILE : 0) +
                                    (newrow >= 0 ? 2 * S::ROW : 0);
             mbar_arrive_expect_tx(bar, bytes);
             if (newrow >= 0) {
-                const TC* kn = reinterpret_cast<const TC*>(p.key) + (size_t)P.s * p.key_stride + (size_t)P.g * D;
-                const TC* vn = reinterpret_cast<const TC*>(p.value) + (size_t)P.s * p.value_stride + (size_t)P.g * D;
+                const TC* kn = reinterpret_cast<const TC*>(p.key) + (size_t)P.s * p.key_stride + (size_t)g * D;
+                const TC* vn = reinterpret_cast<const TC*>(p.value) + (size_t)P.s * p.value_stride + (size_t)g * D;
                 bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW), kn, S::ROW, bar);
                 bulk_g2s(smem_addr(nbuf + (size_t)st * 2 * S::ROW + S::ROW), vn, S::ROW, bar);
             }
             if (newrow == -2) flag_error(p.errors, PKV_DEVERR_SLOT);
             if (first)
-                bulk_g2s(smem_addr(qbuf + qslot_ctr * S::QBYTES),
-                         qg + ((size_t)P.s * p.num_heads + (size_t)P.g * G) * D, S::QBYTES, bar);
+                bulk_g2s(smem_addr(qbuf + qslot_ctr * S::QBYTES), qg + (size_t)m.obase * D, qbytes, bar);
             if (nvalid > 0) {
-                const size_t off = ((size_t)phys * Hkv + P.g) * tile_elems;
+                const size_t off = ((size_t)phys * Hkv + g) * tile_elems;
                 unsigned char* dst = ring + (size_t)st * 2 * S::TILE;
                 bulk_g2s(smem_addr(dst), kc + off, S::TILE, bar);
                 bulk_g2s(smem_addr(dst + S::TILE), vc + off, S::TILE, bar);
@@ -1024,23 +1053,28 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
     uint32_t phase = 0;
     int consumed = 0;
     bool lost = false;
+    // A stage's copies have landed, as seen by every lane; false (for the whole
+    // warp) once the wait gives up.
+    auto stage_ready = [&](uint32_t bar, uint32_t parity) -> bool {
+        return __all_sync(kFull, mbar_wait_bounded(bar, parity, p.wait_limit));
+    };
 
     while (consumed < issued) {
         const uint32_t bar = bar0 + 8 * cons_st;
-        if (!mbar_wait_bounded(bar, phase, kWaitLimit)) {
+        if (!stage_ready(bar, phase)) {
             flag_error(p.errors, PKV_DEVERR_WAIT);
             lost = true;
             break;
         }
         const StageMeta mt = meta[cons_st];
-        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, qscale);
+        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, qscale, mt.nh);
         using Cons = ConsumerFor<TQ, TC, D, BS, G>;
         if constexpr (Cons::kPairs) {
             // the item's next block is in the next stage: take both together
             if (!(mt.flags & kLast) && mt.nvalid > 0 && mt.newrow < 0 && consumed + 1 < issued) {
                 const int st2 = (cons_st + 1 == R) ? 0 : cons_st + 1;
                 const uint32_t ph2 = (cons_st + 1 == R) ? (phase ^ 1u) : phase;
-                if (!mbar_wait_bounded(bar0 + 8 * st2, ph2, kWaitLimit)) {
+                if (!stage_ready(bar0 + 8 * st2, ph2)) {
                     flag_error(p.errors, PKV_DEVERR_WAIT);
                     lost = true;
                     break;
@@ -1074,8 +1108,10 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
                 const int c16 = ch - v * (S::ROW / 16);
                 const uint4 w = reinterpret_cast<const uint4*>(nb + v * S::ROW)[c16];
                 reinterpret_cast<uint4*>(Kt + v * S::TILE + mt.newrow * S::ROW)[c16] = w;
-                TC* cache = const_cast<TC*>(v ? vc : kc);
-                reinterpret_cast<uint4*>(cache + slot_off)[c16] = w;
+                if (mt.flags & kStore) {
+                    TC* cache = const_cast<TC*>(v ? vc : kc);
+                    reinterpret_cast<uint4*>(cache + slot_off)[c16] = w;
+                }
             }
             fence_proxy_async();     // these generic writes precede the stage's next bulk copy
             __syncwarp();
@@ -1091,8 +1127,21 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
         issue();
     }
 
-    // Retire: the last warp to finish resets the scheduling counters.
-    if (!lost && lane == 0) {
+    if (lost) {
+        // Gave up: the copies already issued into this warp's stages still land
+        // before the warp leaves (the CTA's shared memory must outlive them).
+        int st = cons_st;
+        uint32_t ph = phase;
+        for (int k = consumed; k < issued; ++k) {
+            mbar_wait_bounded(bar0 + 8 * st, ph, kWaitLimit);
+            if (++st == R) { st = 0; ph ^= 1u; }
+        }
+        __syncwarp();
+    }
+
+    // Retire, on every path: the last warp to finish resets the scheduling
+    // counters, so the next call on this workspace starts from zero.
+    if (lane == 0) {
         __threadfence();
         const int done = atomicAdd(p.sched + 1, 1);
         if (done == NW - 1) {

@@ -23,6 +23,9 @@ __device__ unsigned int g_device_errors;
 constexpr int kMaxSeqs = 16384;
 constexpr size_t kSchedBytes = 256;
 
+// Polls after which a kernel's bounded wait gives up (pkv_set_wait_limit).
+std::atomic<uint32_t> g_wait_limit{pkv::kWaitLimit};
+
 struct DeviceInfo {
     std::atomic<int> sms{0};
     std::atomic<unsigned int*> errors{nullptr};
@@ -51,13 +54,31 @@ pkv_status device_info(int* sms, unsigned int** errors) {
     return PKV_OK;
 }
 
+// The stream must belong to the current device (the one whose kernels and
+// error word the call uses).  The legacy and per-thread default streams
+// always do.
+pkv_status check_stream(void* stream) {
+    if (stream == nullptr || stream == reinterpret_cast<void*>(cudaStreamLegacy) ||
+        stream == reinterpret_cast<void*>(cudaStreamPerThread))
+        return PKV_OK;
+    int dev = 0, sdev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) {
+        cudaGetLastError();
+        return PKV_ERR_INVALID_ARG;
+    }
+    return sdev == dev ? PKV_OK : PKV_ERR_INVALID_ARG;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int elem_bytes(pkv_dtype t) { return t == PKV_F32 ? 4 : 2; }
 
-bool valid_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+// Query-head columns of one decode work item: the group padded to 1, 2, 4 or
+// 8 (a larger group runs as ceil(G / 8) slices of 8).
+int padded_group(int g) { return g <= 1 ? 1 : g <= 2 ? 2 : g <= 4 ? 4 : 8; }
 
 // Shape checks shared by the workspace query and the launch.
 pkv_status check_shape(int num_seqs, int num_heads, int num_kv_heads, int head_size,
@@ -68,7 +89,6 @@ pkv_status check_shape(int num_seqs, int num_heads, int num_kv_heads, int head_s
     if (head_size != 64 && head_size != 128) return PKV_ERR_UNSUPPORTED;
     if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
     if (num_heads % num_kv_heads != 0) return PKV_ERR_UNSUPPORTED;
-    if (!valid_group(num_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
     if (num_seqs > kMaxSeqs) return PKV_ERR_UNSUPPORTED;
     return PKV_OK;
 }
@@ -215,12 +235,15 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     const WorkspaceLayout wl =
         workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps);
     if (!workspace || !aligned16(workspace) || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
+    if ((st = check_stream(stream)) != PKV_OK) return st;
 
     int sms = 0;
     unsigned int* errors = nullptr;
     if ((st = device_info(&sms, &errors)) != PKV_OK) return st;
 
-    const int G = num_heads / num_kv_heads;
+    const int Greal = num_heads / num_kv_heads;
+    const int G = padded_group(Greal);              // kernel columns per item
+    const int slices = (Greal + G - 1) / G;
     // Shared memory: per-CTA lengths and prefix sums, then one ring per warp.
     const uint32_t seq_smem = (uint32_t)round_up(sizeof(int32_t) * (2 * (size_t)num_seqs + 1), 128);
     // Eight consumer warps per SM hide the per-block latency of the consumer
@@ -278,12 +301,15 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
         p.key_stride = app->key_stride;
         p.value_stride = app->value_stride;
     }
+    p.group = Greal;
+    p.slices = slices;
+    p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
     p.stages = R;
     p.warps = W;
     p.warp_smem = per_warp;
     p.seq_smem = seq_smem;
 
-    const size_t max_items = (size_t)num_seqs * wl.max_parts * num_kv_heads;
+    const size_t max_items = (size_t)num_seqs * wl.max_parts * num_kv_heads * slices;
     size_t ctas = (max_items + W - 1) / W;
     if (ctas > (size_t)sms) ctas = sms;
     const size_t smem = seq_smem + (size_t)W * per_warp;
@@ -402,7 +428,8 @@ pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, 
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = device_info(&sms, &errors);
+    pkv_status st = check_stream(stream);
+    if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::CacheWriteParams p;
     p.key = static_cast<const unsigned char*>(key);
@@ -445,7 +472,8 @@ pkv_status reshape_and_cache_fp8kv(const void* key, const void* value, void* k_c
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = device_info(&sms, &errors);
+    pkv_status st = check_stream(stream);
+    if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::CacheWriteFp8Params p;
     p.key = key;
@@ -489,12 +517,14 @@ pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_lay
     }
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = device_info(&sms, &errors);
+    pkv_status st = check_stream(stream);
+    if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     p.block_mapping = block_mapping;
     p.errors = errors;
     p.block_bytes = block_bytes;
     p.num_blocks = num_blocks;
+    p.num_pairs = num_pairs;
     if (pkv::launch_copy_blocks(p, num_pairs, num_layers, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return PKV_ERR_CUDA;
@@ -534,13 +564,15 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
     if (!reachable(block_mapping)) return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = device_info(&sms, &errors);
+    pkv_status st = check_stream(stream);
+    if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     p.block_mapping = block_mapping;
     p.errors = errors;
     p.block_bytes = block_bytes;
     p.src_blocks = src_num_blocks;
     p.dst_blocks = dst_num_blocks;
+    p.num_pairs = num_pairs;
     if (pkv::launch_swap_blocks(p, num_pairs, num_caches, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return PKV_ERR_CUDA;
@@ -560,7 +592,8 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
     if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
     if (head_size != 64 && head_size != 128) return PKV_ERR_UNSUPPORTED;
     if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
-    if (num_heads % num_kv_heads != 0 || !valid_group(num_heads / num_kv_heads)) return PKV_ERR_UNSUPPORTED;
+    if (num_heads % num_kv_heads != 0 || num_heads / num_kv_heads > pkv::kPrefillMaxGroup)
+        return PKV_ERR_UNSUPPORTED;
     if ((int64_t)num_blocks * num_kv_heads * block_size >= (int64_t)0x7fffffff - block_size)
         return PKV_ERR_UNSUPPORTED;
     if (!(scale > 0.f) || !(scale < INFINITY)) return PKV_ERR_INVALID_ARG;
@@ -573,7 +606,8 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = device_info(&sms, &errors);
+    pkv_status st = check_stream(stream);
+    if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::PrefillArgs a;
     std::memset(&a, 0, sizeof a);
@@ -596,7 +630,14 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.max_query_len = max_query_len;
     a.dtype = dtype;
+    a.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
     return pkv::launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_set_wait_limit(int64_t polls) {
+    if (polls > (int64_t)UINT32_MAX) return PKV_ERR_INVALID_ARG;
+    g_wait_limit.store(polls < 0 ? pkv::kWaitLimit : (uint32_t)polls, std::memory_order_relaxed);
+    return PKV_OK;
 }
 
 pkv_status pkv_read_device_errors(void* stream, uint32_t* bits) {

@@ -1,5 +1,6 @@
 // Paged prefill launch: tensor maps for q and the two caches, one kernel
-// instance per (element type, head size, block size, group size).
+// instance per (element type, head size, block size); the group size is a
+// launch parameter.
 #include <atomic>
 #include <cstring>
 
@@ -17,9 +18,12 @@ bool encode(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* ba
     return encode_tiled(map, type, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS>
 pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
-    using S = PrefillShape<T, D, BS, G>;
+    using S = PrefillShape<T, D, BS>;
+    const int G = a.num_heads / a.num_kv_heads;
+    if (G < 1 || G > kPrefillMaxGroup) return PKV_ERR_UNSUPPORTED;
+    const int QT = S::M / G;                 // queries per query tile
     const CUtensorMapDataType type =
         std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const cuuint64_t esz = sizeof(T);
@@ -27,7 +31,7 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     {
         const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)a.num_heads, (cuuint64_t)a.num_tokens};
         const cuuint64_t strides[2] = {D * esz, (cuuint64_t)a.num_heads * D * esz};
-        const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)S::QT};
+        const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)QT};
         if (!encode(&tm_q, type, 3, a.q, dims, strides, box)) return PKV_ERR_CUDA;
     }
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
@@ -53,7 +57,10 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     p.num_kv_heads = a.num_kv_heads;
     p.num_blocks = a.num_blocks;
     p.max_blocks_per_seq = a.max_blocks_per_seq;
-    p.q_tiles = (a.max_query_len + S::CQ - 1) / S::CQ;
+    p.group = G;
+    p.qt = QT;
+    p.wait_limit = a.wait_limit;
+    p.q_tiles = (a.max_query_len + 2 * QT - 1) / (2 * QT);
     p.cache_rows = (int)rows;
     // scheduling groups: as many (sequence, KV head) pairs as keep their K/V
     // (at the longest possible context) within half of L2
@@ -63,11 +70,11 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
             return PKV_ERR_CUDA;
         const double pair_bytes = (double)a.max_blocks_per_seq * BS * D * sizeof(T) * 2.0;
         const double fit = (l2 / 2.0) / (pair_bytes > 1.0 ? pair_bytes : 1.0);
-        p.group = fit < 1.0 ? 1 : (fit > 4096.0 ? 4096 : (int)fit);
+        p.sched_group = fit < 1.0 ? 1 : (fit > 4096.0 ? 4096 : (int)fit);
     }
     const int64_t grid = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
     if (grid > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
-    auto kernel = paged_prefill_kernel<T, D, BS, G>;
+    auto kernel = paged_prefill_kernel<T, D, BS>;
     static std::atomic<bool> configured[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
@@ -83,22 +90,11 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     return PKV_OK;
 }
 
-template <typename T, int D, int BS>
-pkv_status by_group(const PrefillArgs& a, cudaStream_t stream) {
-    switch (a.num_heads / a.num_kv_heads) {
-        case 1: return run<T, D, BS, 1>(a, stream);
-        case 2: return run<T, D, BS, 2>(a, stream);
-        case 4: return run<T, D, BS, 4>(a, stream);
-        case 8: return run<T, D, BS, 8>(a, stream);
-        default: return PKV_ERR_UNSUPPORTED;
-    }
-}
-
 template <typename T, int D>
 pkv_status by_block(const PrefillArgs& a, cudaStream_t stream) {
     switch (a.block_size) {
-        case 16: return by_group<T, D, 16>(a, stream);
-        case 32: return by_group<T, D, 32>(a, stream);
+        case 16: return run<T, D, 16>(a, stream);
+        case 32: return run<T, D, 32>(a, stream);
         default: return PKV_ERR_UNSUPPORTED;
     }
 }

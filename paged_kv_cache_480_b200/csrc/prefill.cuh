@@ -21,7 +21,12 @@ struct PrefillArgs {
     int num_tokens, num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks;
     int max_blocks_per_seq, max_query_len;
     pkv_dtype dtype;
+    uint32_t wait_limit;   // polls before a bounded wait gives up
 };
+
+// Largest group (query heads per KV head) of the prefill kernel: one query
+// tile of 128 rows holds 128 / G queries of G heads each.
+constexpr int kPrefillMaxGroup = 128;
 
 // Encodes the tensor maps and launches; PKV_ERR_UNSUPPORTED for shapes with
 // no kernel, PKV_ERR_CUDA if the driver's tensor-map encoder or the launch fails.

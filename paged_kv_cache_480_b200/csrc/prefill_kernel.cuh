@@ -10,7 +10,9 @@
 // CTA = (sequence, KV head g, two query tiles of M = 128 rows each); a row
 // is a (query, head-of-group) pair, row = query * G + head, so every K/V
 // tile serves the G query heads that share it, and both query tiles of the
-// CTA share each K/V tile brought into shared memory.  Roles:
+// CTA share each K/V tile brought into shared memory.  A query tile holds
+// QT = floor(128 / G) queries; when G does not divide 128 its last
+// 128 - QT * G rows are zero and never written out.  Roles:
 //   warps 0-3 and 4-7  softmax of query tile 0 and 1, one row per thread
 //                      (warp w reaches tensor-memory lanes 32(w%4) .. +31);
 //   warp 8             issues the MMAs (one thread);
@@ -91,8 +93,8 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // Bounded wait taken by all 32 lanes; true only if every lane saw the phase,
 // so a failure leaves the whole warp on the same path.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
-    const bool got = mbar_wait_bounded(bar, parity, kWaitLimit);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+    const bool got = mbar_wait_bounded(bar, parity, limit);
     return __all_sync(kAll, got);
 }
 
@@ -106,8 +108,11 @@ struct PrefillParams {
     unsigned int* errors;
     float scale_log2;                 // softmax scale * log2(e), > 0
     int num_tokens, num_seqs, num_heads, num_kv_heads, num_blocks, max_blocks_per_seq;
+    int group;                        // G = num_heads / num_kv_heads, 1 .. 128
+    int qt;                           // queries per query tile: floor(128 / G)
+    uint32_t wait_limit;              // polls before a wait for progress gives up
     int q_tiles;                      // CTAs (query-tile pairs) per (sequence, KV head)
-    int group;                        // (sequence, KV head) pairs per scheduling group, >= 1
+    int sched_group;                  // (sequence, KV head) pairs per scheduling group, >= 1
     int cache_rows;                   // rows of the [NB * Hkv * bs][D] view of a cache
 };
 
@@ -119,11 +124,9 @@ struct PrefillParams {
 #define PKV_PREFILL_VST128 2
 #endif
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS>
 struct PrefillShape {
     static constexpr int M = 128;               // rows per query tile
-    static constexpr int QT = M / G;            // queries per query tile
-    static constexpr int CQ = 2 * QT;           // queries per CTA
     static constexpr int N = 128;               // keys per tile
     static constexpr int DH = D / 64;           // 64-dim halves (one 128-byte swizzle row each)
     static constexpr int BPT = N / BS;          // cache blocks per key tile
@@ -149,11 +152,11 @@ struct PrefillShape {
 
 constexpr uint32_t kPrefillThreads = 352;
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
-    using S = PrefillShape<T, D, BS, G>;
+    using S = PrefillShape<T, D, BS>;
     using namespace prefill;
     constexpr int KST = S::KST, VST = S::VST;
     constexpr int N = S::N;
@@ -164,15 +167,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     unsigned char* smem = smem_raw + pad;
     const uint32_t sm = raw_s + pad;                // 1024-byte aligned shared address
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.group, QT = p.qt, CQ = 2 * QT;  // heads per KV head; queries per tile and per CTA
+    const int QROWS = QT * G;                       // rows of a query tile that hold queries
+    const uint32_t wl = p.wait_limit;
 
     griddep_wait();
     // ---- which queries: the later ones (more keys) are scheduled first ----
     const int Hkv = p.num_kv_heads;
     const int pairs = p.num_seqs * Hkv;
-// groups of p.group (sequence, KV head) pairs, one after the other; inside
+    // groups of p.sched_group (sequence, KV head) pairs, one after the other; inside
     // a group the tiles with most keys go first.  The host sizes groups so
     // that a group's K/V fits in half of L2 while its query tiles read it.
-    const int gp = min(p.group, pairs);
+    const int gp = min(p.sched_group, pairs);
     const int per_group = gp * p.q_tiles;
     const int grp = (int)blockIdx.x / per_group;
     const int in_g = (int)blockIdx.x - grp * per_group;
@@ -184,16 +190,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int q0 = p.query_start_loc[s];
     const int n = p.query_start_loc[s + 1] - q0;
     const int L = p.context_lens[s];
-    const int i0 = tile * S::CQ;
-    if (n < 0 || n > L || n > p.q_tiles * S::CQ || L > p.max_blocks_per_seq * BS || q0 < 0 ||
+    const int i0 = tile * CQ;
+    if (n < 0 || n > L || n > p.q_tiles * CQ || L > p.max_blocks_per_seq * BS || q0 < 0 ||
         q0 + n > p.num_tokens) {
         if (threadIdx.x == 0) flag_error(p.errors, PKV_DEVERR_CONTEXT);
         return;
     }
     if (i0 >= n) return;                            // whole CTA, before any barrier or TMEM use
     // key tiles each query tile needs (0: the tile holds no query)
-    const int nT0 = (L - n + min(i0 + S::QT, n) + N - 1) / N;
-    const int nT1 = i0 + S::QT < n ? (L - n + min(i0 + S::CQ, n) + N - 1) / N : 0;
+    const int nT0 = (L - n + min(i0 + QT, n) + N - 1) / N;
+    const int nT1 = i0 + QT < n ? (L - n + min(i0 + CQ, n) + N - 1) / N : 0;
     auto nTx = [&](int x) { return x ? nT1 : nT0; };
     const bool two = nT1 > 0;
     const int nT = max(nT0, nT1);
@@ -254,12 +260,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ===================== TMA producers: warp 9 Q and K, warp 10 V =====================
         const bool is_v = warp == 10;
         int issued = 0;
+        if (!is_v && QROWS < S::M) {
+            // rows past the tile's queries take zeros (they are never written
+            // out; zeros keep their softmax finite and off the redo path)
+            const int nz = (S::M - QROWS) * 8;          // 16-byte chunks per 64-dim half
+            for (int c = lane; c < (two ? 2 : 1) * S::DH * nz; c += 32) {
+                const int x = c / (S::DH * nz), rem = c - x * S::DH * nz;
+                const int dh = rem / nz, k = rem - dh * nz;
+                *reinterpret_cast<uint4*>(smem + x * S::Q_BYTES + dh * S::Q_HALF + QROWS * 128 + k * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async();   // visible to the tensor core's reads of Q
+            __syncwarp();
+        }
         if (lane == 0) {
             if (!is_v) {
-                mbar_arrive_expect_tx(bar_q, (two ? 2 : 1) * S::Q_BYTES);
+                mbar_arrive_expect_tx(bar_q, (uint32_t)((two ? 2 : 1) * S::DH * QROWS * 128));
                 for (int x = 0; x < (two ? 2 : 1); ++x)
                     for (int dh = 0; dh < S::DH; ++dh)
-                        tc05::tma_load_3d(q_base(x) + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0 + x * S::QT,
+                        tc05::tma_load_3d(q_base(x) + dh * S::Q_HALF, &tm_q, dh * 64, g * G, q0 + i0 + x * QT,
                                           bar_q);
             }
             const int nst = is_v ? VST : KST;
@@ -269,7 +288,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const uint32_t empty = is_v ? bar_vempty(st) : bar_kempty(st);
                 const uint32_t full = is_v ? bar_vfull(st) : bar_kfull(st);
                 const uint32_t dst = is_v ? v_base(st) : k_base(st);
-                if (t >= nst && !mbar_wait_bounded(empty, ((t / nst) - 1) & 1, kWaitLimit)) {
+                if (t >= nst && !mbar_wait_bounded(empty, ((t / nst) - 1) & 1, wl)) {
                     flag_error(p.errors, PKV_DEVERR_WAIT);
                     break;
                 }
@@ -297,7 +316,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         issued = __shfl_sync(kAll, issued, 0);
         if (is_v && need_vz && issued == nT) {
             const int st = (nT - 1) % VST;
-            if (warp_wait(bar_vfull(st), ((nT - 1) / VST) & 1)) {
+            if (warp_wait(bar_vfull(st), ((nT - 1) / VST) & 1, wl)) {
                 const int rows = vz_r1 - vz_r0;
                 for (int c = lane; c < rows * S::DH * 8; c += 32) {   // 16-byte chunks
                     const int dh = c / (rows * 8);
@@ -320,7 +339,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint64_t dq = tc05::smem_desc(q_base(0), 16, 1024);
             const uint64_t dk = tc05::smem_desc(k_base(0), 16, 1024);
             const uint64_t dv = tc05::smem_desc(v_base(0), S::KV_HALF, 1024);
-            bool ok = mbar_wait_bounded(bar_q, 0, kWaitLimit);
+            bool ok = mbar_wait_bounded(bar_q, 0, wl);
             bool vz_seen = !need_vz;
             auto qk = [&](int x, int i) {                    // S_x = Q_x K_i^T
                 const uint32_t d = tm + x * S::TM_TILE + S::TM_S;
@@ -337,12 +356,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             };
             auto pv = [&](int x, int i) -> bool {            // O_x += P_x V_i
                 const int sv = i % VST;
-                if (!mbar_wait_bounded(bar_vfull(sv), (i / VST) & 1, kWaitLimit)) return false;
+                if (!mbar_wait_bounded(bar_vfull(sv), (i / VST) & 1, wl)) return false;
                 if (i == nT - 1 && !vz_seen) {
-                    if (!mbar_wait_bounded(bar_vz, 0, kWaitLimit)) return false;
+                    if (!mbar_wait_bounded(bar_vz, 0, wl)) return false;
                     vz_seen = true;
                 }
-                if (!mbar_wait_bounded(bar_p(x), i & 1, kWaitLimit)) return false;
+                if (!mbar_wait_bounded(bar_p(x), i & 1, wl)) return false;
                 tc05::fence_after_sync();
                 const uint32_t base = tm + x * S::TM_TILE;
                 const uint64_t vd = dv + (uint64_t)((sv * S::KV_BYTES) >> 4);
@@ -355,7 +374,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 return true;
             };
             for (int i = 0; ok && i < nT; ++i) {
-                if (!mbar_wait_bounded(bar_kfull(i % KST), (i / KST) & 1, kWaitLimit)) { ok = false; break; }
+                if (!mbar_wait_bounded(bar_kfull(i % KST), (i / KST) & 1, wl)) { ok = false; break; }
                 tc05::fence_after_sync();
                 if (i < nT0) qk(0, i);
                 if (two && i >= 1) {                         // V(i-1) last read by PV_1(i-1)
@@ -386,8 +405,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             bool ok = true;
             const int wq = warp & 3;
             const int r = wq * 32 + lane;               // row within the tile
-            const int qi = i0 + x * S::QT + r / G;      // query of this row
-            const bool valid = qi < n;
+            const int qi = i0 + x * QT + r / G;         // query of this row
+            const bool valid = r < QROWS && qi < n;
             // keys 0 .. pos are visible.  Rows past the sequence's queries are
             // never written and every row's softmax is its own, so they take no
             // mask (a mask there would turn every tile of their warp diagonal)
@@ -396,7 +415,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const float sl2 = p.scale_log2;
             float m_ref = -INFINITY, l = 0.f;           // reference max (log2 units), sum of weights
             for (int i = 0; i < nTme; ++i) {
-                if (!warp_wait(bar_s(x), i & 1)) { ok = false; break; }
+                if (!warp_wait(bar_s(x), i & 1, wl)) { ok = false; break; }
                 tc05::fence_after_sync();
                 const int key0 = i * N;
                 const bool diag = __any_sync(kAll, key0 + N - 1 > pos);   // a diagonal (or past-the-end) tile
@@ -575,7 +594,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 mbar_arrive(bar_p(x));
             }
             // ---- epilogue: O / l to the output ----
-            if (ok && warp_wait(bar_o(x), 0)) {
+            if (ok && warp_wait(bar_o(x), 0, wl)) {
                 tc05::fence_after_sync();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 T* orow = reinterpret_cast<T*>(p.out) +

@@ -21,6 +21,12 @@ Five named workloads (base seed 480 + index):
                  filled and shared); each sample then generates U{0..256}
                  tokens of its own (a scenario, see make_cow_scenario).
 
+One more shape beyond those five, for multi-query attention (every query
+head shares one KV head):
+
+  mqa_long_bf16  gqa_long_bf16's sequences and lengths with 64 query heads
+                 over a single KV head (seed 480 + 7).
+
 Every slot of the pool that holds no context token is filled with NaN, so a
 kernel that reads past a sequence's length or into a free block shows it.
 The new token of a decode step (position context_len - 1) is not in the
@@ -45,6 +51,8 @@ CONFIGS = {
                           block_size=16, dtype="bf16"),
     "cow_bf16": dict(index=4, num_seqs=512, num_heads=32, num_kv_heads=32, head_size=128,
                      block_size=16, dtype="bf16"),
+    "mqa_long_bf16": dict(index=7, num_seqs=16, num_heads=64, num_kv_heads=1, head_size=128,
+                          block_size=16, dtype="bf16"),
 }
 
 DTYPE_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
@@ -150,7 +158,7 @@ def make_layout(name, block_size=None, seed=None, num_seqs=None, max_context=Non
         lens = rng.integers(256, 2049, S)
     elif name == "llama7b_bf16":
         lens = np.clip(np.round(np.exp(math.log(700.0) + 0.8 * rng.standard_normal(S))), 16, 4096)
-    elif name == "gqa_long_bf16":
+    elif name in ("gqa_long_bf16", "mqa_long_bf16"):
         lens = rng.integers(16384, 32769, S)
     elif name == "cow_bf16":
         raise ValueError("cow_bf16 is a scenario: use make_cow_scenario")

@@ -81,3 +81,36 @@ def test_copy_blocks_bad_pair_is_flagged():
     assert pkv.read_device_errors() & 8
     assert torch.equal(k[2].view(torch.int16), before[1].view(torch.int16))
     assert torch.equal(k[3].view(torch.int16), before[3].view(torch.int16))
+
+
+def test_copy_blocks_overlapping_pairs_are_skipped_and_flagged():
+    """Pairs whose result would depend on the order of the copies (a
+    destination that is another pair's source, two pairs with one
+    destination) are skipped and set PKV_DEVERR_COPY_OVERLAP; the other pairs,
+    including several that share one source, are copied as the oracle copies
+    them."""
+    gen = torch.Generator(device="cuda").manual_seed(35)
+    k = _rand_raw((16, 2, 16, 64), "bf16", gen)
+    v = _rand_raw((16, 2, 16, 64), "bf16", gen)
+    mapping = np.array([[1, 2], [2, 3],          # chain: 2 is a destination and a source
+                        [4, 5], [6, 5],          # one destination twice
+                        [7, 8], [7, 9], [10, 11]], np.int64)   # clean (one shared source)
+    clean = mapping[4:]
+    host = [raw(k, "bf16"), raw(v, "bf16")]
+    oracle.copy_blocks(host, clean)
+    pkv.copy_blocks([k], [v], torch.from_numpy(mapping).cuda())
+    assert pkv.read_device_errors() == 32
+    assert same_bits(raw(k, "bf16"), host[0]) and same_bits(raw(v, "bf16"), host[1])
+
+
+def test_swap_blocks_repeated_destination_is_skipped_and_flagged():
+    gen = torch.Generator(device="cuda").manual_seed(36)
+    kd = _rand_raw((8, 2, 16, 64), "f16", gen)
+    kh = torch.zeros((6, 2, 16, 64), dtype=torch.float16).pin_memory()
+    mapping = np.array([[0, 1], [3, 1], [2, 4]], np.int64)     # pool-to-pool: a source may equal a destination id
+    ref = raw(kh, "f16")
+    oracle.swap_blocks([raw(kd, "f16")], [ref], mapping[2:])
+    pkv.swap_blocks([kd], [kh], torch.from_numpy(mapping).cuda())
+    torch.cuda.synchronize()
+    assert pkv.read_device_errors() == 32
+    assert same_bits(raw(kh, "f16"), ref)

@@ -23,6 +23,32 @@ pytestmark = pytest.mark.gpu
 BF16_NAN = 0x7fc0
 
 
+def check_cache_contents(cache, host, gpu_tables, model_tables, lens, bs, chunk=512):
+    """Every sequence's keys (or values) read through the GPU manager's table
+    equal, bit for bit, those read through the model's table from the oracle's
+    pool: each GPU block pairs with one model block, and their rows holding
+    context tokens are identical."""
+    pair_rows = {}
+    for s, L in enumerate(lens):
+        for j in range(-(-int(L) // bs)):
+            key = (int(gpu_tables[s, j]), int(model_tables[s, j]))
+            pair_rows[key] = max(pair_rows.get(key, 0), min(bs, int(L) - j * bs))
+    gb = np.array([k[0] for k in pair_rows], np.int64)
+    mb = np.array([k[1] for k in pair_rows], np.int64)
+    nv = np.array(list(pair_rows.values()), np.int64)
+    assert len(np.unique(gb)) == len(gb) and len(np.unique(mb)) == len(mb), "blocks pair up one to one"
+    dev_host = torch.from_numpy(host.view(np.int16))
+    cache16 = cache.view(torch.int16)
+    for a in range(0, len(gb), chunk):
+        g = torch.from_numpy(gb[a:a + chunk]).to(cache.device)
+        m = torch.from_numpy(mb[a:a + chunk])
+        got = cache16[g]                                   # [n, Hkv, bs, D]
+        want = dev_host[m].to(cache.device)
+        rows = torch.arange(bs, device=cache.device)[None, :] < torch.from_numpy(nv[a:a + chunk]).to(cache.device)[:, None]
+        bad = (got != want).any(dim=-1) & rows[:, None, :]
+        assert not bad.any().item(), f"{int(bad.sum())} cache rows differ"
+
+
 def run_scenario(sc):
     dev = "cuda"
     NB, Hkv, bs, D = sc.num_blocks, sc.num_kv_heads, sc.block_size, sc.head_size
@@ -74,6 +100,8 @@ def run_scenario(sc):
     mt = np.full((sc.num_seqs, MB), -1, np.int32)
     for s in seqs:
         mt[s, :len(model.tables[s])] = model.tables[s]
+    check_cache_contents(kc, hk, gt, mt, lens, bs)
+    check_cache_contents(vc, hv, gt, mt, lens, bs)
     q = wl.cow_queries(sc, dev)
     out = torch.empty_like(q)
     pkv.paged_attention_decode(out, q, kc, vc, torch.from_numpy(gt).to(dev),

@@ -84,6 +84,13 @@ def test_gqa_long_bf16():
     check_step(lay, rel_bar=2e-2)
 
 
+def test_mqa_long_bf16():
+    """64 query heads over one KV head at 16K-32K tokens: eight 8-head slices
+    per KV head, split contexts and the merge."""
+    lay = wl.make_layout("mqa_long_bf16")
+    check_step(lay, rel_bar=2e-2)
+
+
 # ---------------------------------------------------------------------------
 # edge cases at small sizes
 # ---------------------------------------------------------------------------
@@ -93,7 +100,7 @@ EDGE_LENS = [0, 1, 15, 16, 17, 255, 256, 257, 511, 512, 513, 1000, 33]
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [16, 32])
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 8, 16, 64])
 def test_edge_lengths(dtype, D, bs, G):
     Hkv = 2
     lay = wl.custom_layout(dtype, num_heads=Hkv * G, num_kv_heads=Hkv, head_size=D, block_size=bs,
@@ -210,3 +217,38 @@ def test_context_beyond_bound_is_flagged():
                                max_context_len=32)
     assert pkv.read_device_errors() & 4
     assert torch.equal(out[0], torch.zeros_like(out[0]))
+
+
+# ---------------------------------------------------------------------------
+# bounded waits that run out: the call reports it, the next call is whole
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("G", [1, 8, 16])
+def test_wait_limit_gives_up_then_next_call_is_exact(G):
+    """With the wait limit at 0 every wait for a stage's copies gives up at
+    once: the call returns, sets PKV_DEVERR_WAIT and leaves the workspace's
+    counters at zero, so the next normal call on the same workspace matches
+    the oracle element by element."""
+    lay = wl.custom_layout("bf16", 2 * G, 2, 128, 16, [700, 1300, 90, 1, 0, 513], seed=40 + G)
+    ten = wl.make_tensors(lay, device="cuda", pending_new_token=False)
+    host = host_copy(ten, "bf16")
+    ref = oracle_step(lay, host, write_new=False)
+    need = pkv.paged_attention_workspace_size(lay.num_seqs, lay.num_heads, 2, 128, 16, 1300, 2, 0)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    bt = torch.from_numpy(lay.block_tables).cuda()
+    cl = torch.from_numpy(lay.context_lens).cuda()
+    out = torch.empty_like(ten["q"])
+    assert pkv.read_device_errors() == 0
+    try:
+        pkv.set_wait_limit(0)
+        pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                                   max_context_len=1300, workspace=ws)
+        bits = pkv.read_device_errors()
+    finally:
+        pkv.set_wait_limit(-1)
+    assert bits & 16, bits
+    assert torch.count_nonzero(ws[:256]).item() == 0     # counters reset on the give-up path too
+    out.fill_(float("nan"))
+    pkv.paged_attention_decode(out, ten["q"], ten["k_cache"], ten["v_cache"], bt, cl, lay.scale,
+                               max_context_len=1300, workspace=ws)
+    assert pkv.read_device_errors() == 0
+    compare(out, ref, "bf16")

@@ -61,10 +61,17 @@ def test_fp8_step_matches_oracle(name, kw):
 
 @pytest.mark.parametrize("dtype,G,D,bs", [("bf16", 8, 128, 16), ("bf16", 4, 64, 32), ("f16", 8, 64, 16),
                                           ("f16", 1, 128, 32), ("bf16", 2, 64, 16), ("f32", 8, 128, 16),
-                                          ("f32", 1, 64, 32)])
+                                          ("f32", 1, 64, 32), ("bf16", 3, 128, 16), ("f16", 3, 64, 32),
+                                          ("f32", 3, 128, 16), ("bf16", 16, 128, 16), ("f16", 16, 128, 32),
+                                          ("bf16", 64, 128, 16), ("f32", 64, 64, 16)])
 def test_fp8_edge_lengths(dtype, G, D, bs):
     lay = wl.custom_layout(dtype, 2 * G, 2, D, bs, [0, 1, 15, 16, 17, 255, 257, 513, 1000], seed=60 + G + D)
     _check(lay)
+
+
+def test_fp8_mqa_long():
+    """The MQA workload's shape (64 query heads over one KV head) over E4M3 caches."""
+    _check(wl.make_layout("mqa_long_bf16", num_seqs=4))
 
 
 def test_fp8_forced_partitions():

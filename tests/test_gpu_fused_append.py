@@ -49,7 +49,9 @@ def test_fused_append_matches_oracle_and_two_call_path(name, kw, ps):
 
 
 @pytest.mark.parametrize("dtype,G,D,bs", [("bf16", 8, 128, 16), ("f16", 4, 64, 32), ("f32", 1, 128, 16),
-                                          ("bf16", 2, 128, 32)])
+                                          ("bf16", 2, 128, 32), ("bf16", 3, 128, 16), ("f32", 3, 64, 16),
+                                          ("bf16", 16, 128, 16), ("f16", 16, 64, 32), ("bf16", 64, 128, 16),
+                                          ("f16", 64, 128, 32)])
 def test_fused_append_edge_lengths(dtype, G, D, bs):
     lens = [0, 1, 15, 16, 17, 255, 256, 257, 513, 1000]
     lay = wl.custom_layout(dtype, 2 * G, 2, D, bs, lens, seed=40 + G)
@@ -59,6 +61,7 @@ def test_fused_append_edge_lengths(dtype, G, D, bs):
     assert err == 0
     ref = oracle_step(lay, host)
     assert same_bits(raw(ten["k_cache"], dtype), host["k_cache"])
+    assert same_bits(raw(ten["v_cache"], dtype), host["v_cache"])
     compare(out, ref, dtype)
 
 

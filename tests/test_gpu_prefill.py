@@ -52,6 +52,11 @@ CASES = [
     ("bf16", 4, 4, 128, 16, [128, 256, 64], [128, 256, 64]),         # exact multiples of the tiles
     ("bf16", 8, 8, 128, 16, [2000], [700]),                          # the K/V ring wraps many times
     ("f16", 16, 2, 64, 16, [777, 400], [300, 399]),                  # G = 8, D = 64
+    ("bf16", 6, 2, 128, 16, [300, 90, 47], [300, 45, 47]),            # G = 3: 42 queries, 2 zero rows per tile
+    ("f16", 15, 3, 64, 32, [260, 129], [100, 129]),                  # G = 5: 25 queries, 3 zero rows
+    ("bf16", 32, 2, 128, 16, [500, 17, 9], [40, 17, 1]),             # G = 16: 8 queries per tile
+    ("f16", 64, 1, 128, 32, [300, 70], [9, 5]),                      # G = 64 (MQA): 2 queries per tile
+    ("bf16", 128, 1, 64, 16, [200, 3], [4, 3]),                      # G = 128: 1 query per tile
 ]
 
 
@@ -205,3 +210,23 @@ def test_prefill_full_size_sampled(name):
     ref = oracle.paged_attention(q_rows, raw(ten["k_cache"], lay.dtype), raw(ten["v_cache"], lay.dtype),
                                  tables, lens, lay.scale, lay.dtype, lay.num_kv_heads, lay.block_size)
     compare(out[torch.from_numpy(rows).cuda()], ref, lay.dtype)
+
+
+@pytest.mark.parametrize("G", [1, 3, 16])
+def test_prefill_wait_limit_gives_up_then_next_call_is_exact(G):
+    """With the wait limit at 0 every role's first wait gives up: the call
+    returns with PKV_DEVERR_WAIT set (each role lets its copies land, the MMA
+    role waits for its issued products, the tensor memory is freed), and the
+    next normal call matches the oracle."""
+    lay = _layout("bf16", 2 * G, 2, 128, 16, [300, 40, 129], [300, 7, 129], seed=8 + G)
+    ten = wl.make_prefill_tensors(lay, device="cuda")
+    assert pkv.read_device_errors() == 0
+    try:
+        pkv.set_wait_limit(0)
+        _, bits = _gpu(lay, ten)
+    finally:
+        pkv.set_wait_limit(-1)
+    assert bits & 16, bits
+    out, err = _gpu(lay, ten)
+    assert err == 0
+    compare(out, _oracle(lay, ten), "bf16")

@@ -68,7 +68,10 @@ def test_partition_and_workspace_sizes(lib):
     # partials: S * parts * H * (D floats + an (m, l) pair), parts at the smallest size
     assert big >= 64 * 16 * 40 * (128 * 4 + 8)
     assert lib.paged_attention_workspace_size(64, 40, 7, 128, 16, 2048, 1, 0) == 0   # G not integral
-    assert lib.paged_attention_workspace_size(64, 48, 4, 128, 16, 2048, 1, 0) == 0   # G = 12
+    # any integral group: G = 12 (slices of 8 + 4 heads) and MQA (G = 64) need the same
+    # partials per query head as MHA
+    assert lib.paged_attention_workspace_size(64, 48, 4, 128, 16, 2048, 1, 0) >= 64 * 8 * 48 * (128 * 4 + 8)
+    assert lib.paged_attention_workspace_size(64, 64, 1, 128, 16, 2048, 1, 0) >= 64 * 8 * 64 * (128 * 4 + 8)
     assert lib.paged_attention_workspace_size(64, 40, 40, 96, 16, 2048, 1, 0) == 0   # head_size 96
 
 
@@ -131,7 +134,7 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _prefill(lib, dtype=0) == 2               # f32: no tensor-core kernel
     assert _prefill(lib, d=96) == 2                  # head size
     assert _prefill(lib, bs=8) == 2                  # block size
-    assert _prefill(lib, h=12, hkv=1) == 2           # G = 12
+    assert _prefill(lib, h=256, hkv=1) == 2          # G = 256: a query tile holds at most 128 rows
     assert _prefill(lib, q=8) == 1                   # misaligned q
     assert _prefill(lib, qsl=18) == 1                # misaligned int32 array
     assert _prefill(lib, mq=41) == 1                 # bound above the token count
@@ -141,3 +144,9 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _prefill(lib, scale=0.0) == 1
     assert _prefill(lib, nb=1 << 27, hkv=4) == 2     # pool rows beyond 2^31
     assert _prefill(lib, t=0, mq=0) == 0             # nothing to do
+
+
+def test_wait_limit_setting(lib):
+    assert lib.pkv_set_wait_limit(0) == 0
+    assert lib.pkv_set_wait_limit(1 << 33) == 1      # beyond 32 bits
+    assert lib.pkv_set_wait_limit(-1) == 0           # back to the default
