@@ -101,8 +101,9 @@ const char* pkv_version(void);
  *                  num_kv_heads, any value: MHA, GQA and MQA)
  *   block_size     tokens per block, 16 or 32
  *   num_seqs ... max_blocks_per_seq   the sizes above
- *   max_context_len host-known upper bound of context_lens (> 0); sizes the
- *                  workspace and picks the split
+ *   max_context_len host-known upper bound of context_lens; sizes the
+ *                  workspace and picks the split.  0 means max_blocks_per_seq
+ *                  * block_size (the workspace must then be sized for that)
  *   dtype          element type of q, caches and out (all the same)
  *   partition_size tokens per split-context partition: 0 = library choice
  *                  (a per-call size between 8 and 16 blocks, 16 and 32

@@ -3,7 +3,17 @@
 // unnormalised accumulator acc_p, the running max m_p (log2 units) and the
 // sum l_p, the exact identity
 //   M = max_p m_p,  w_p = 2^(m_p - M),  out = sum_p w_p acc_p / sum_p w_p l_p
-// gives the attention over the whole context.
+// gives the attention over the whole context.  Partials with m_p = -inf
+// (no key) are skipped.
+//
+// Two layouts of the partials.  The CUDA-core decode numbers them through
+// per-sequence prefix sums it publishes (a sequence with one partition wrote
+// its output itself).  The tensor-core decode splits the key tiles of all
+// units (sequence, KV head, slice of up to 128 query heads) into equal
+// contiguous ranges, one per CTA; CTA c writes two partials (one per half)
+// for unit u in slots 2 * (c + u) and 2 * (c + u) + 1, rows [slot * rows, +
+// rows).  The CTAs whose range meets unit u follow from the per-sequence
+// prefix sums of key tiles it publishes.
 #pragma once
 
 #include "common.cuh"
@@ -12,11 +22,16 @@ namespace pkv {
 
 struct ReduceParams {
     void* out;
-    const float* part_acc;     // [items][G][D]
-    const float2* part_ml;     // [items][G]
-    const int32_t* prefix;     // [S + 1] partitions before each sequence
+    const float* part_acc;     // [partials][H][D]
+    const float2* part_ml;     // [partials][H]
+    const int32_t* prefix;     // [S + 1] partitions before each sequence (CUDA-core decode)
     int num_seqs, num_heads, num_kv_heads;
-    int max_parts;             // partitions per sequence at most
+    int max_parts;             // partials per sequence at most
+    // tensor-core decode (tc_prefix non-null): tc_prefix[s] = key tiles of one
+    // unit before sequence s, [S] = their total; tc_ctas CTAs, tc_slices
+    // units per KV head, tc_rows rows per slot
+    const int32_t* tc_prefix;
+    int tc_ctas, tc_slices, tc_rows;
 };
 
 __device__ __forceinline__ float merge_ex2(float x) {
@@ -37,13 +52,41 @@ __global__ void __launch_bounds__(128) lse_merge_kernel(const ReduceParams p) {
     __shared__ float4 s_num[NPG][TPH];
     griddep_wait();
     const int s = blockIdx.x, h = blockIdx.y;
-    const int np = p.prefix[s + 1] - p.prefix[s];
-    if (np <= 1) return;                // written by the decode kernel itself
-    const int G = p.num_heads / p.num_kv_heads;
-    const int g = h / G, hh = h % G;
-    const int base = p.prefix[s];
-    for (int q = threadIdx.x; q < np; q += blockDim.x)
-        s_ml[q] = p.part_ml[((size_t)(base + q) * p.num_kv_heads + g) * G + hh];
+    int np;
+    size_t base, rs, ro;                // partial q sits at row (base + q) * rs + ro
+    int64_t tc_first = 0, tc_tiles = 0; // tensor-core decode: first CTA of the unit, tiles of all units
+    if (p.tc_prefix != nullptr) {
+        const int G = p.num_heads / p.num_kv_heads;
+        const int g = h / G, hh = h - g * G, sl = hh / 128;
+        const int NU = p.num_kv_heads * p.tc_slices;
+        const int u = g * p.tc_slices + sl;
+        const int64_t Ts = p.tc_prefix[s + 1] - p.tc_prefix[s];
+        tc_tiles = (int64_t)p.tc_prefix[p.num_seqs] * NU;
+        int64_t cl = -1;
+        if (Ts > 0) {
+            // the CTA whose range [floor(c T / C), floor((c + 1) T / C)) holds tile t
+            const int64_t C = p.tc_ctas;
+            const int64_t gu = (int64_t)p.tc_prefix[s] * NU + (int64_t)u * Ts;
+            tc_first = ((gu + 1) * C - 1) / tc_tiles;
+            cl = ((gu + Ts) * C - 1) / tc_tiles;
+        }
+        np = 2 * (int)(cl - tc_first + 1);
+        base = 2 * ((size_t)tc_first + (size_t)s * NU + u);
+        rs = p.tc_rows;
+        ro = hh - sl * 128;
+    } else {
+        np = p.prefix[s + 1] - p.prefix[s];
+        if (np <= 1) return;            // written by the decode kernel itself
+        base = p.prefix[s];
+        rs = p.num_heads;
+        ro = h;
+    }
+    for (int q = threadIdx.x; q < np; q += blockDim.x) {
+        // with fewer tiles than CTAs some CTAs' ranges are empty: they wrote nothing
+        const int64_t c = tc_first + q / 2, C = p.tc_ctas;
+        const bool written = p.tc_prefix == nullptr || (c + 1) * tc_tiles / C > c * tc_tiles / C;
+        s_ml[q] = written ? p.part_ml[(base + q) * rs + ro] : make_float2(-INFINITY, 0.f);
+    }
     __syncthreads();
     float M = -INFINITY, den = 0.f;
     for (int q = 0; q < np; ++q) M = fmaxf(M, s_ml[q].x);
@@ -53,8 +96,8 @@ __global__ void __launch_bounds__(128) lse_merge_kernel(const ReduceParams p) {
 
     const int pg = threadIdx.x / TPH, d4 = threadIdx.x % TPH;
     const float4* acc = reinterpret_cast<const float4*>(p.part_acc) + d4;
-    const size_t stride = (size_t)p.num_kv_heads * G * TPH;           // float4s between partitions
-    const size_t first = (((size_t)base * p.num_kv_heads + g) * G + hh) * TPH;
+    const size_t stride = rs * TPH;                                   // float4s between partials
+    const size_t first = (base * rs + ro) * TPH;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
         for (int q0 = pg; q0 < np; q0 += 4 * NPG) {

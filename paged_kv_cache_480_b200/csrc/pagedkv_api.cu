@@ -6,6 +6,7 @@
 
 #include "cache_ops.cuh"
 #include "decode_launch.cuh"
+#include "decode_tc.cuh"
 #include "pagedkv.h"
 #include "prefill.cuh"
 
@@ -120,19 +121,26 @@ struct WorkspaceLayout {
     int max_parts;
 };
 
+// Whether a plain decode call takes the tensor-core split-context kernel:
+// 16-bit q and caches, at least kDecodeTcMinGroup query heads per KV head,
+// and the library's choice of partitions.
+bool use_decode_tc(int num_heads, int num_kv_heads, int dtype, int partition_size) {
+    return dtype != PKV_F32 && num_heads / num_kv_heads >= pkv::kDecodeTcMinGroup && partition_size == 0;
+}
+
 WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_size,
-                                 int max_context_len, int ps) {
+                                 int max_context_len, int ps, bool tc = false) {
     WorkspaceLayout w;
     const int ctx = max_context_len > 0 ? max_context_len : 1;
     w.max_parts = (ctx + ps - 1) / ps;
-    const int G = num_heads / num_kv_heads;
-    const size_t items = (size_t)num_seqs * w.max_parts * num_kv_heads;
+    size_t rows = w.max_parts > 1 ? (size_t)num_seqs * w.max_parts * num_heads : 0;   // partial rows
+    if (tc) rows = pkv::decode_tc_partial_rows(num_seqs, num_heads, num_kv_heads);
     w.prefix = kSchedBytes;
     size_t off = round_up(w.prefix + sizeof(int32_t) * (num_seqs + 1), 256);
     w.part_ml = off;
-    if (w.max_parts > 1) off = round_up(off + items * G * sizeof(float2), 256);
+    off = round_up(off + rows * sizeof(float2), 256);
     w.part_acc = off;
-    if (w.max_parts > 1) off = round_up(off + items * G * head_size * sizeof(float), 256);
+    off = round_up(off + rows * head_size * sizeof(float), 256);
     w.total = off;
     return w;
 }
@@ -188,7 +196,12 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_he
     const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
                                      partition_size);
     if (ps == 0) return 0;
-    return workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps).total;
+    // room for either decode kernel (the fused and FP8 variants take the CUDA-core one)
+    const size_t a = workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps).total;
+    if (!use_decode_tc(num_heads, num_kv_heads, dtype, partition_size)) return a;
+    const size_t b =
+        workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps, true).total;
+    return a > b ? a : b;
 }
 
 pkv_status paged_attention_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
@@ -224,6 +237,7 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     if (st != PKV_OK) return st;
     if (num_blocks <= 0 || max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
     if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * block_size) return PKV_ERR_INVALID_ARG;
+    if (max_context_len == 0) max_context_len = max_blocks_per_seq * block_size;   // the table's bound
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned4(block_tables) || !aligned4(context_lens))
         return PKV_ERR_INVALID_ARG;
@@ -232,14 +246,43 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
                                      partition_size, &ps_hi);
     if (ps == 0) return PKV_ERR_INVALID_ARG;
+    const bool tc = !fp8_cache && app == nullptr && use_decode_tc(num_heads, num_kv_heads, dtype, partition_size);
     const WorkspaceLayout wl =
-        workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps);
+        workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps, tc);
     if (!workspace || !aligned16(workspace) || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
     if ((st = check_stream(stream)) != PKV_OK) return st;
 
     int sms = 0;
     unsigned int* errors = nullptr;
     if ((st = device_info(&sms, &errors)) != PKV_OK) return st;
+
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    if (tc) {
+        pkv::DecodeTcArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.out = out;
+        a.q = q;
+        a.k_cache = k_cache;
+        a.v_cache = v_cache;
+        a.block_tables = block_tables;
+        a.context_lens = context_lens;
+        a.errors = errors;
+        a.prefix = reinterpret_cast<int32_t*>(ws + wl.prefix);
+        a.part_acc = reinterpret_cast<float*>(ws + wl.part_acc);
+        a.part_ml = reinterpret_cast<float2*>(ws + wl.part_ml);
+        a.scale = scale;
+        a.num_seqs = num_seqs;
+        a.num_heads = num_heads;
+        a.num_kv_heads = num_kv_heads;
+        a.head_size = head_size;
+        a.block_size = block_size;
+        a.num_blocks = num_blocks;
+        a.max_blocks_per_seq = max_blocks_per_seq;
+        a.max_context_len = max_context_len;
+        a.dtype = dtype;
+        a.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+        return pkv::launch_decode_tc(a, static_cast<cudaStream_t>(stream));
+    }
 
     const int Greal = num_heads / num_kv_heads;
     const int G = padded_group(Greal);              // kernel columns per item
@@ -269,7 +312,6 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     if (fp8_mma && 32 * W > PKV_FP8_THREADS) W = PKV_FP8_THREADS / 32;
     if (W < 1) return PKV_ERR_UNSUPPORTED;
 
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
     pkv::DecodeParams p{};
     p.out = out;
     p.q = q;
@@ -331,7 +373,7 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     }
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (wl.max_parts > 1) {
-        pkv::ReduceParams r;
+        pkv::ReduceParams r{};   // zero: no fixed-stride layout (prefix sums)
         r.out = out;
         r.part_acc = p.part_acc;
         r.part_ml = p.part_ml;
@@ -431,7 +473,7 @@ pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, 
     pkv_status st = check_stream(stream);
     if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
-    pkv::CacheWriteParams p;
+    pkv::CacheWriteParams p{};
     p.key = static_cast<const unsigned char*>(key);
     p.value = static_cast<const unsigned char*>(value);
     p.k_cache = static_cast<unsigned char*>(k_cache);
@@ -475,7 +517,7 @@ pkv_status reshape_and_cache_fp8kv(const void* key, const void* value, void* k_c
     pkv_status st = check_stream(stream);
     if (st == PKV_OK) st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
-    pkv::CacheWriteFp8Params p;
+    pkv::CacheWriteFp8Params p{};
     p.key = key;
     p.value = value;
     p.k_cache = static_cast<unsigned char*>(k_cache);

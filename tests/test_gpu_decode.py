@@ -28,7 +28,8 @@ def _lib():
 # keys whose logits jump far above the rest of the context
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("name,ps", [("llama7b_bf16", 0), ("gqa_long_bf16", 0), ("gqa_long_bf16", 512),
-                                     ("opt13b_f16", 0), ("tiny_mha_f32", 16)])
+                                     ("opt13b_f16", 0), ("tiny_mha_f32", 16), ("mqa_long_bf16", 0),
+                                     ("mqa_long_bf16", 512)])
 def test_decode_logit_jumps(name, ps):
     """Unit-variance inputs with the keys of random context positions scaled
     by 8: single keys dominate their rows, wherever they fall in a slice,
@@ -105,6 +106,15 @@ def test_edge_lengths(dtype, D, bs, G):
     Hkv = 2
     lay = wl.custom_layout(dtype, num_heads=Hkv * G, num_kv_heads=Hkv, head_size=D, block_size=bs,
                            context_lens=EDGE_LENS, seed=7 + G + D + bs)
+    check_step(lay)
+
+
+@pytest.mark.parametrize("dtype,H,D,bs", [("bf16", 256, 128, 16), ("f16", 160, 64, 32), ("bf16", 130, 128, 32)])
+def test_groups_beyond_128_heads(dtype, H, D, bs):
+    """One KV head for more than 128 query heads: slices of 128 rows on the
+    tensor cores (the last slice partly filled)."""
+    lay = wl.custom_layout(dtype, num_heads=H, num_kv_heads=1, head_size=D, block_size=bs,
+                           context_lens=[0, 1, 17, 255, 256, 257, 1000, 2049], seed=70 + H)
     check_step(lay)
 
 
