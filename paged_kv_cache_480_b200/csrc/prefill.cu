@@ -13,6 +13,25 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Item counters of the persistent prefill grid: each launch takes the next of
+// kCounterSlots pairs (item counter, finished CTAs), which its last CTA
+// resets to zero.  Up to kCounterSlots launches may run at the same time.
+constexpr int kCounterSlots = 64;
+__device__ int g_prefill_sched[2 * kCounterSlots];
+std::atomic<unsigned> g_prefill_launches{0};
+std::atomic<int*> g_prefill_sched_addr[kMaxDevices];
+
+int* counter_slot(int dev) {
+    int* base = g_prefill_sched_addr[dev].load(std::memory_order_acquire);
+    if (base == nullptr) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_prefill_sched) != cudaSuccess || addr == nullptr) return nullptr;
+        base = static_cast<int*>(addr);
+        g_prefill_sched_addr[dev].store(base, std::memory_order_release);
+    }
+    return base + 2 * (g_prefill_launches.fetch_add(1, std::memory_order_relaxed) % kCounterSlots);
+}
+
 bool encode(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const cuuint64_t* dims,
             const cuuint64_t* strides_bytes, const cuuint32_t* box) {
     return encode_tiled(map, type, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -72,12 +91,17 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
         const double fit = (l2 / 2.0) / (pair_bytes > 1.0 ? pair_bytes : 1.0);
         p.sched_group = fit < 1.0 ? 1 : (fit > 4096.0 ? 4096 : (int)fit);
     }
-    const int64_t grid = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
-    if (grid > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+    const int64_t items = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
+    if (items > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
     auto kernel = paged_prefill_kernel<T, D, BS>;
     static std::atomic<bool> configured[kMaxDevices];
-    int dev = 0;
+    int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PKV_ERR_CUDA;
+    // persistent: one CTA per SM (fewer if there are fewer items)
+    const int64_t grid = items < sms ? items : sms;
+    p.sched = counter_slot(dev);
+    if (p.sched == nullptr) return PKV_ERR_CUDA;
     if (!configured[dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) !=
             cudaSuccess)
