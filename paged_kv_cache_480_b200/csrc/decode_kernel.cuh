@@ -1066,8 +1066,20 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
             lost = true;
             break;
         }
-        const StageMeta mt = meta[cons_st];
-        if (mt.flags & kFirst) cons.begin(qbuf + mt.qslot * S::QBYTES, qscale, mt.nh);
+        // Over an FP8 cache (threads capped at 128 registers) only what the block
+        // needs is held in registers and finish() reads the item's output rows
+        // from the stage's metadata; the 16-bit kernels keep a copy (measured:
+        // each way is the faster one for its kernel).
+        constexpr bool kLean = std::is_same<TC, fp8e4m3>::value;
+        StageMeta mt;
+        if constexpr (kLean) {
+            mt.flags = meta[cons_st].flags;
+            mt.nvalid = meta[cons_st].nvalid;
+            mt.newrow = meta[cons_st].newrow;
+        } else {
+            mt = meta[cons_st];
+        }
+        if (mt.flags & kFirst) cons.begin(qbuf + meta[cons_st].qslot * S::QBYTES, qscale, meta[cons_st].nh);
         using Cons = ConsumerFor<TQ, TC, D, BS, G>;
         if constexpr (Cons::kPairs) {
             // the item's next block is in the next stage: take both together
@@ -1079,12 +1091,12 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
                     lost = true;
                     break;
                 }
-                const StageMeta mt2 = meta[st2];
-                if (mt2.nvalid > 0 && mt2.newrow < 0) {
+                const int nvalid2 = meta[st2].nvalid;
+                if (nvalid2 > 0 && meta[st2].newrow < 0) {
                     const unsigned char* Ka = ring + (size_t)cons_st * 2 * S::TILE;
                     const unsigned char* Kb = ring + (size_t)st2 * 2 * S::TILE;
-                    cons.block2(Ka, Ka + S::TILE, mt.nvalid, Kb, Kb + S::TILE, mt2.nvalid, qscale);
-                    if (mt2.flags & kLast) cons.finish(mt2, p);
+                    cons.block2(Ka, Ka + S::TILE, mt.nvalid, Kb, Kb + S::TILE, nvalid2, qscale);
+                    if (meta[st2].flags & kLast) cons.finish(meta[st2], p);
                     __syncwarp();
                     consumed += 2;
                     cons_st = st2;
@@ -1101,14 +1113,15 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
             // (it holds the slot's old bytes) and into the cache slot.
             unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
             const unsigned char* nb = nbuf + (size_t)cons_st * 2 * S::ROW;
-            const size_t slot_off = (size_t)mt.slot / BS * Hkv * tile_elems +
-                                    (size_t)mt.g * tile_elems + (size_t)(mt.slot % BS) * D;
+            const int64_t slot = meta[cons_st].slot;
+            const size_t slot_off = (size_t)slot / BS * Hkv * tile_elems +
+                                    (size_t)meta[cons_st].g * tile_elems + (size_t)(slot % BS) * D;
             for (int ch = lane; ch < 2 * S::ROW / 16; ch += 32) {
                 const int v = ch >= S::ROW / 16;
                 const int c16 = ch - v * (S::ROW / 16);
                 const uint4 w = reinterpret_cast<const uint4*>(nb + v * S::ROW)[c16];
                 reinterpret_cast<uint4*>(Kt + v * S::TILE + mt.newrow * S::ROW)[c16] = w;
-                if (mt.flags & kStore) {
+                if (meta[cons_st].flags & kStore) {
                     TC* cache = const_cast<TC*>(v ? vc : kc);
                     reinterpret_cast<uint4*>(cache + slot_off)[c16] = w;
                 }
@@ -1120,7 +1133,10 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
             const unsigned char* Kt = ring + (size_t)cons_st * 2 * S::TILE;
             cons.block(Kt, Kt + S::TILE, mt.nvalid, qscale);
         }
-        if (mt.flags & kLast) cons.finish(mt, p);
+        if (mt.flags & kLast) {
+            if constexpr (kLean) cons.finish(meta[cons_st], p);
+            else cons.finish(mt, p);
+        }
         __syncwarp();
         ++consumed;
         if (++cons_st == R) { cons_st = 0; phase ^= 1u; }

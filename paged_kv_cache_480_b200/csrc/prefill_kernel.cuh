@@ -466,10 +466,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 };
                 if (!mbar_wait_bounded(bar_qfull(0), qx[0] & 1, wl)) { ok = false; break; }
                 ++qx[0];
-                if (two) {
-                    if (!mbar_wait_bounded(bar_qfull(1), qx[1] & 1, wl)) { ok = false; break; }
-                    ++qx[1];
-                }
                 for (int i = 0; ok && i < nT; ++i) {
                     const int jt = jt0 + i;
                     if (!mbar_wait_bounded(bar_kfull(jt % KST), (jt / KST) & 1, wl)) { ok = false; break; }
@@ -479,7 +475,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         if (!pv(1, i - 1)) { ok = false; break; }
                         tc05::commit(bar_vempty((jt - 1) % VST));
                     }
-                    if (i < nT1) qk(1, i);
+                    if (i < nT1) {
+                        if (i == 0) {                           // q tile 1 is needed from here on
+                            if (!mbar_wait_bounded(bar_qfull(1), qx[1] & 1, wl)) { ok = false; break; }
+                            ++qx[1];
+                        }
+                        qk(1, i);
+                    }
                     tc05::commit(bar_kempty(jt % KST));
                     if (i < nT0) {
                         if (!pv(0, i)) { ok = false; break; }
