@@ -269,7 +269,7 @@ def kernel_source_sha():
 
 def prefill_source_sha():
     h = hashlib.sha256()
-    for f in ("prefill_kernel.cuh", "prefill.cu", "tc05.cuh", "common.cuh"):
+    for f in ("prefill_kernel.cuh", "prefill.cu", "tc05.cuh", "tc_softmax.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_480_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
