@@ -33,7 +33,8 @@
  *   Streams  GPU calls are asynchronous on the given cudaStream_t (passed as
  *            void*, NULL = the legacy default stream); they never
  *            synchronise, except pkv_read_device_errors.  The stream must
- *            belong to the current device (PKV_ERR_INVALID_ARG otherwise).
+ *            belong to the current device (not checked: the call's kernels,
+ *            scratch and error word are the current device's).
  *   Errors   argument errors are found on the host before anything is
  *            launched and return a status with nothing launched.  A failed
  *            launch returns PKV_ERR_CUDA.  Conditions only the device can see
@@ -288,7 +289,8 @@ pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_lay
  *
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.
+ * before any stream capture.  The stream must belong to the current device,
+ * whose array the call uses (not checked).
  *
  * Sharing: every call, on every stream and thread, uses the same array, which
  * keeps the previous call's contents.  Calls that overlap on the GPU race on

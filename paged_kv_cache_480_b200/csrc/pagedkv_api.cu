@@ -55,22 +55,6 @@ pkv_status device_info(int* sms, unsigned int** errors) {
     return PKV_OK;
 }
 
-// The stream must belong to the current device (the one whose kernels and
-// error word the call uses).  The legacy and per-thread default streams
-// always do.
-pkv_status check_stream(void* stream) {
-    if (stream == nullptr || stream == reinterpret_cast<void*>(cudaStreamLegacy) ||
-        stream == reinterpret_cast<void*>(cudaStreamPerThread))
-        return PKV_OK;
-    int dev = 0, sdev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
-    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) {
-        cudaGetLastError();
-        return PKV_ERR_INVALID_ARG;
-    }
-    return sdev == dev ? PKV_OK : PKV_ERR_INVALID_ARG;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -250,7 +234,6 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     const WorkspaceLayout wl =
         workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps, tc);
     if (!workspace || !aligned16(workspace) || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
-    if ((st = check_stream(stream)) != PKV_OK) return st;
 
     int sms = 0;
     unsigned int* errors = nullptr;
@@ -470,8 +453,7 @@ pkv_status reshape_and_cache(const void* key, const void* value, void* k_cache, 
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = check_stream(stream);
-    if (st == PKV_OK) st = device_info(&sms, &errors);
+    pkv_status st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::CacheWriteParams p{};
     p.key = static_cast<const unsigned char*>(key);
@@ -514,8 +496,7 @@ pkv_status reshape_and_cache_fp8kv(const void* key, const void* value, void* k_c
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = check_stream(stream);
-    if (st == PKV_OK) st = device_info(&sms, &errors);
+    pkv_status st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::CacheWriteFp8Params p{};
     p.key = key;
@@ -559,8 +540,7 @@ pkv_status copy_blocks(void* const* k_caches, void* const* v_caches, int num_lay
     }
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = check_stream(stream);
-    if (st == PKV_OK) st = device_info(&sms, &errors);
+    pkv_status st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     p.block_mapping = block_mapping;
     p.errors = errors;
@@ -606,8 +586,7 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
     if (!reachable(block_mapping)) return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = check_stream(stream);
-    if (st == PKV_OK) st = device_info(&sms, &errors);
+    pkv_status st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     p.block_mapping = block_mapping;
     p.errors = errors;
@@ -648,8 +627,7 @@ pkv_status paged_attention_prefill(void* out, const void* q, const void* k_cache
         return PKV_ERR_INVALID_ARG;
     int sms = 0;
     unsigned int* errors = nullptr;
-    pkv_status st = check_stream(stream);
-    if (st == PKV_OK) st = device_info(&sms, &errors);
+    pkv_status st = device_info(&sms, &errors);
     if (st != PKV_OK) return st;
     pkv::PrefillArgs a;
     std::memset(&a, 0, sizeof a);
