@@ -7,11 +7,12 @@
 // weights; P = 2^(S * scale*log2e - m_ref) rounded to the element type.  Most
 // tiles keep every row's reference and take one sweep; m_ref is raised (O
 // and l rescaled) only when a logit rises more than 8 above it, so O stays
-// exact up to the final division by l.  The P of keys 0-63 lands on S
-// columns 0-31 and is held in registers until one warp vote finds no jump
-// there (a jump redoes the tile from the intact S); keys 64-127 are stored at
-// once and voted after (a jump there rescales the stored P and O and
-// recomputes them from their intact S).
+// exact up to the final division by l.  A row's first tile takes the
+// largest of its first 8 logits as the starting reference.  The P of keys
+// 0-63 lands on S columns 0-31 and is held in registers until one warp vote
+// finds no jump there (a jump redoes the tile from the intact S); keys
+// 64-127 are stored at once and voted after (a jump there rescales the
+// stored P and O and recomputes them from their intact S).
 #pragma once
 
 #include <math.h>
@@ -140,6 +141,21 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int key0,
     // overwrites S chunks 0 and 1 only; S chunks 2 and 3 stay intact.
     float l_add = 0.f, alpha = 1.f;
     bool full = !__all_sync(kAll, m_ref != -INFINITY);
+    if (full && __all_sync(kAll, m_ref == -INFINITY)) {
+        // every row's first tile: the reference starts at the largest of its
+        // first 8 logits, and the sweep below raises it where needed (a
+        // causal or context-end mask hides a suffix of the keys, so a row
+        // that sees none of these sees nothing in the tile and keeps -inf)
+        uint32_t v8[8];
+        tc05::tmem_ld8(ts, v8);
+        tc05::tmem_wait_ld();
+        float m8 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (key0 + c <= pos) m8 = fmaxf(m8, __uint_as_float(v8[c]));
+        m_ref = m8 * sl2;                           // the scale is positive
+        full = !__all_sync(kAll, m_ref != -INFINITY);
+    }
     if (!full) {
         // Most tiles keep every row's reference: one sweep at it.  The P
         // of chunks 0 and 1 is held until no row of the warp has a logit
@@ -212,8 +228,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t ts, uint32_t to, int key0,
         }
     }
     if (full) {
-        // a row's first tile (or rows that have seen only masked keys, or
-        // a jump in chunk 0 or 1): the row maximum first
+        // rows that have seen only masked keys, or a jump in chunk 0 or 1:
+        // the row maximum first
         float mx = -INFINITY;
 #pragma unroll
         for (int hh = 0; hh < N / 64; ++hh) {
