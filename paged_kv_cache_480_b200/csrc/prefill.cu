@@ -81,23 +81,29 @@ pkv_status run(const PrefillArgs& a, cudaStream_t stream) {
     p.wait_limit = a.wait_limit;
     p.q_tiles = (a.max_query_len + 2 * QT - 1) / (2 * QT);
     p.cache_rows = (int)rows;
-    // scheduling groups: as many (sequence, KV head) pairs as keep their K/V
-    // (at the longest possible context) within half of L2
+    int dev = 0, sms = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    // Scheduling groups of (sequence, KV head) pairs.  Each CTA holds about
+    // 1.5 items (the one it runs and the one it claimed ahead), so the K/V in
+    // flight is that of (1.5 * CTAs + the group's items) / (items per pair)
+    // pairs; the group is as large as keeps that within 3/4 of L2 at the
+    // longest possible context, and at least 2 pairs.  Large groups let the
+    // heaviest-first order inside a group balance the CTAs (whole prompts of
+    // mixed lengths); small ones keep a pair's items close in time, so its
+    // K/V comes from DRAM about once (chunks of long contexts).
     {
-        int dev = 0, l2 = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
-            return PKV_ERR_CUDA;
         const double pair_bytes = (double)a.max_blocks_per_seq * BS * D * sizeof(T) * 2.0;
-        const double fit = (l2 / 2.0) / (pair_bytes > 1.0 ? pair_bytes : 1.0);
-        p.sched_group = fit < 1.0 ? 1 : (fit > 4096.0 ? 4096 : (int)fit);
+        const double in_flight = 0.75 * l2 / (pair_bytes > 1.0 ? pair_bytes : 1.0);
+        const double g = in_flight - 1.5 * sms / (p.q_tiles > 0 ? p.q_tiles : 1);
+        p.sched_group = g < 2.0 ? 2 : (g > 4096.0 ? 4096 : (int)g);
     }
     const int64_t items = (int64_t)p.q_tiles * a.num_seqs * a.num_kv_heads;
     if (items > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
     auto kernel = paged_prefill_kernel<T, D, BS>;
     static std::atomic<bool> configured[kMaxDevices];
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PKV_ERR_CUDA;
     // persistent: one CTA per SM (fewer if there are fewer items)
     const int64_t grid = items < sms ? items : sms;
     p.sched = counter_slot(dev);
