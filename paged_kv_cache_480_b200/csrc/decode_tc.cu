@@ -82,6 +82,7 @@ pkv_status run(const DecodeTcArgs& a, cudaStream_t stream) {
     r.tc_ctas = kDecodeTcCtas;
     r.tc_slices = p.slices;
     r.tc_rows = GR;
+    r.tc_unit_cost = kTcUnitCost;
     cudaError_t e = std::is_same<T, __nv_bfloat16>::value ? merge_bf16(r, D, stream) : merge_f16(r, D, stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

@@ -12,10 +12,11 @@
 //
 // Work: a unit is (sequence s, KV head g, slice of up to 128 of its query
 // heads); its keys form ceil(L / 128) tiles of N = 128 keys.  The tiles of all
-// units, in order, are split into equal contiguous ranges, one per CTA of a
-// grid of kDecodeTcCtas persistent CTAs (one per SM).  A CTA streams its range
-// without a break at unit boundaries: the K/V rings and the tensor-core
-// pipeline run on across units, q is double-buffered per unit.
+// units, in order, are split into contiguous ranges of equal cost, one per CTA
+// of a grid of kDecodeTcCtas persistent CTAs (one per SM); a unit costs its
+// tiles plus kTcUnitCost for its start and its partial write.  A CTA streams
+// its range without a break at unit boundaries: the K/V rings and the
+// tensor-core pipeline run on across units, q is double-buffered per unit.
 //
 // Rows of the M = 128 tile are the unit's heads (rows past them hold zeros and
 // are never written out).  The CTA's tiles alternate between two halves x =
@@ -47,11 +48,15 @@ namespace pkv {
 // CTAs of the tensor-core decode: one per SM of a B200.  The work split and
 // the partial-result layout depend on it, not on the device the call runs on.
 constexpr int kDecodeTcCtas = 148;
+// The cost of a unit's start and partial write in key tiles (measured: a CTA
+// whose range meets two units ends about two tiles' time later than one
+// whose range meets one).
+constexpr int kTcUnitCost = 2;
 
 struct DecodeTcParams {
     float* part_acc;                  // [2 * (ctas + units)][rows][D] unnormalised O
     float2* part_ml;                  // [2 * (ctas + units)][rows] (m_ref in log2 units, l)
-    int32_t* prefix;                  // [S + 1] key tiles of one unit before each sequence (CTA 0 writes)
+    int32_t* prefix;                  // [S + 1] cost of one unit of each earlier sequence, summed (CTA 0 writes)
     const int32_t* block_tables;      // [S][MB]
     const int32_t* context_lens;      // [S]
     unsigned int* errors;
@@ -107,33 +112,34 @@ __device__ __forceinline__ int tc_seq_len(const DecodeTcParams& p, int s) {
 }
 
 // Walk over the segments of a CTA's range: maximal runs of consecutive tiles
-// of one unit.  Every role walks the same sequence independently.
+// of one unit.  Every role walks the same sequence independently.  Costs are
+// counted in the range's own units: the unit's kTcUnitCost, then its tiles.
 struct TcSegWalk {
     int s, u, t;       // sequence, unit within the sequence, next tile of that unit
     int L, Ts;         // the sequence's length and tiles per unit
-    int left;          // tiles of the range not yet handed out
+    int left;          // cost from the unit's first tile to the end of the CTA's range
     int NU;            // units per sequence
     // Next segment: unit (s, u), tiles [t0, t0 + n).  False at the range's end.
     __device__ __forceinline__ bool next(const DecodeTcParams& p, int& ss, int& uu, int& t0, int& n, int& LL,
                                          int& TT) {
-        if (left <= 0) return false;
-        while (t >= Ts) {
+        while (t >= Ts) {                           // unit done (or empty): the next one
+            if (Ts > 0) left -= Ts + kTcUnitCost;
             t = 0;
             if (++u == NU) {
                 u = 0;
-                ++s;
+                if (++s >= p.num_seqs) return false;
                 L = tc_seq_len(p, s);
                 Ts = (L + 127) / 128;
             }
         }
-        n = min(Ts - t, left);
+        if (t >= left) return false;
+        n = min(Ts - t, left - t);
         ss = s;
         uu = u;
         t0 = t;
         LL = L;
         TT = Ts;
         t += n;
-        left -= n;
         return true;
     }
 };
@@ -198,6 +204,11 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         mbar_init(bar_fin, 1);
         fence_mbar_init();
     }
+    if (threadIdx.x == 32) {
+        tc05::prefetch_tmap(&tm_q);
+        tc05::prefetch_tmap(&tm_k);
+        tc05::prefetch_tmap(&tm_v);
+    }
     if (warp == 0) {
         tc05::tmem_alloc(smem_addr(tm_holder), S::TM_COLS);
         tc05::tmem_relinquish();
@@ -216,10 +227,12 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
     griddep_wait();
     griddep_launch();                               // the merge kernel may get resident; it waits for us
 
-    // ---- the CTA's range: tiles [start(c), start(c + 1)), start(c) = floor(c * total / C), of the
-    // NU * sum_s tiles(s) tiles of all units ----
-    // pass 1: T; pass 2: find the sequence holding the range's first tile
-    // (CTA 0 also publishes the per-sequence prefix sums for the merge).
+    // ---- the CTA's range: [floor(c V / C), floor((c + 1) V / C)) of the cost
+    // index, V = NU * sum_s w(s), w(s) = kTcUnitCost + tiles(s) for a sequence
+    // with keys, else 0; the unit (s, u) spans [NU W(s) + u w(s), + w(s)) with
+    // W(s) = sum of w over earlier sequences, its tiles the last tiles(s) of it.
+    // pass 1: V; pass 2: find the sequence holding the range's start (CTA 0
+    // also publishes W for the merge).
     auto block_sum = [&](int v) -> int {            // all threads; returns the block total
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kAll, v, off);
@@ -230,27 +243,38 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         __syncthreads();
         return tot;
     };
+    // the block tables to L2 while the lengths are summed (a slice per CTA)
+    if (warp == 10) {
+        const uint32_t lines = (uint32_t)(((int64_t)p.num_seqs * p.max_blocks_per_seq + 31) / 32);
+        const uint32_t per = (lines + C - 1) / C, hi = min(lines, (uint32_t)(c + 1) * per);
+        for (uint32_t i = (uint32_t)c * per + lane; i < hi; i += 32)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.block_tables + (size_t)i * 32));
+    }
+    int w_first = 0;                                // this thread's w in the first chunk
     int64_t total = 0;
     for (int base = 0; base < p.num_seqs; base += nthreads) {
         const int s = base + threadIdx.x;
-        int L = 0;
+        int w = 0;
         if (s < p.num_seqs) {
             const int raw = __ldg(p.context_lens + s);
-            L = tc_seq_len(p, s);
+            const int L = tc_seq_len(p, s);
             if (c == 0 && L != raw) flag_error(p.errors, PKV_DEVERR_CONTEXT);
+            w = L > 0 ? (L + 127) / 128 + kTcUnitCost : 0;
         }
-        total += block_sum((L + 127) / 128);
+        if (base == 0) w_first = w;
+        total += block_sum(w);
     }
-    const int64_t tiles_all = total * NU;
-    const int64_t g0 = tiles_all * c / C, g1 = tiles_all * (c + 1) / C;
+    const int64_t vtot = total * NU;
+    const int64_t v0 = vtot * c / C, v1 = vtot * (c + 1) / C;
     if (threadIdx.x == 0) scratch[16] = -1;
     __syncthreads();
     {
         int64_t carry = 0;
         for (int base = 0; base < p.num_seqs; base += nthreads) {
             const int s = base + threadIdx.x;
-            const int ts = s < p.num_seqs ? (tc_seq_len(p, s) + 127) / 128 : 0;
-            int incl = ts;                          // inclusive scan over the block
+            int w = w_first;
+            if (base > 0) w = s < p.num_seqs && tc_seq_len(p, s) > 0 ? (tc_seq_len(p, s) + 127) / 128 + kTcUnitCost : 0;
+            int incl = w;                           // inclusive scan over the block
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int v = __shfl_up_sync(kAll, incl, off);
@@ -259,16 +283,17 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
             if (lane == 31) scratch[warp] = incl;
             __syncthreads();
             int before = 0, chunk = 0;
-            for (int w = 0; w < nwarps; ++w) {
-                if (w < warp) before += scratch[w];
-                chunk += scratch[w];
+            for (int wp = 0; wp < nwarps; ++wp) {
+                if (wp < warp) before += scratch[wp];
+                chunk += scratch[wp];
             }
-            const int64_t pre = carry + before + incl - ts;    // tiles of one unit before sequence s
+            const int64_t pre = carry + before + incl - w;    // W(s)
             if (s < p.num_seqs) {
                 if (c == 0) p.prefix[s] = (int32_t)pre;
-                if (ts > 0 && pre * NU <= g0 && g0 < (pre + ts) * NU) {
+                if (w > 0 && pre * NU <= v0 && v0 < (pre + w) * NU) {
                     scratch[16] = s;
-                    scratch[17] = (int)(g0 - pre * NU);         // offset of the first tile in s's units
+                    scratch[17] = (int)(v0 - pre * NU);         // offset of the start in s's units
+                    scratch[18] = (int)pre;
                 }
             }
             carry += chunk;
@@ -278,18 +303,21 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         if (c == 0 && threadIdx.x == 0) p.prefix[p.num_seqs] = (int32_t)carry;
     }
     __syncthreads();
-    const int range = (int)(g1 - g0);
     TcSegWalk walk0;
-    walk0.left = range;
     walk0.NU = NU;
-    if (range > 0) {
+    bool has_work = false;
+    if (v1 > v0 && scratch[16] >= 0) {
         walk0.s = scratch[16];
         walk0.L = tc_seq_len(p, walk0.s);
         walk0.Ts = (walk0.L + 127) / 128;
-        walk0.u = scratch[17] / walk0.Ts;
-        walk0.t = scratch[17] - walk0.u * walk0.Ts;
+        const int w = walk0.Ts + kTcUnitCost, o = scratch[17];
+        walk0.u = o / w;
+        walk0.t = max(0, o - walk0.u * w - kTcUnitCost);
+        // the range ends at most one range length past the unit's first tile
+        walk0.left = (int)(v1 - ((int64_t)scratch[18] * NU + (int64_t)walk0.u * w + kTcUnitCost));
+        has_work = walk0.t < walk0.left;
     } else {
-        walk0.s = walk0.u = walk0.t = walk0.L = walk0.Ts = 0;
+        walk0.s = walk0.u = walk0.t = walk0.L = walk0.Ts = walk0.left = 0;
     }
     tc05::fence_before_sync();
     __syncthreads();
@@ -300,8 +328,8 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
     auto k_base = [&](int st) { return sm + S::OFF_K + (uint32_t)st * S::KV_BYTES; };
     auto v_base = [&](int st) { return sm + S::OFF_V + (uint32_t)st * S::KV_BYTES; };
 
-    if (range <= 0) {
-        // no tile (fewer tiles than CTAs): nothing to do
+    if (!has_work) {
+        // no tile in the range (more CTAs than work): nothing to do
     } else if (warp >= 9) {
         // ===================== TMA producers: warp 9 q and K, warp 10 V =====================
         const bool is_v = warp == 10;

@@ -197,6 +197,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_init(bar_fin, 1);
         fence_mbar_init();
     }
+    if (threadIdx.x == 32) {
+        tc05::prefetch_tmap(&tm_q);
+        tc05::prefetch_tmap(&tm_k);
+        tc05::prefetch_tmap(&tm_v);
+    }
     if (warp == 0) {
         tc05::tmem_alloc(smem_addr(tm_holder), S::TM_COLS);
         tc05::tmem_relinquish();
