@@ -231,8 +231,7 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
     // index, V = NU * sum_s w(s), w(s) = kTcUnitCost + tiles(s) for a sequence
     // with keys, else 0; the unit (s, u) spans [NU W(s) + u w(s), + w(s)) with
     // W(s) = sum of w over earlier sequences, its tiles the last tiles(s) of it.
-    // pass 1: V; pass 2: find the sequence holding the range's start (CTA 0
-    // also publishes W for the merge).
+    // CTA 0 also publishes W for the merge.
     auto block_sum = [&](int v) -> int {            // all threads; returns the block total
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kAll, v, off);
@@ -250,30 +249,63 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
         for (uint32_t i = (uint32_t)c * per + lane; i < hi; i += 32)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(p.block_tables + (size_t)i * 32));
     }
-    int w_first = 0;                                // this thread's w in the first chunk
-    int64_t total = 0;
-    for (int base = 0; base < p.num_seqs; base += nthreads) {
-        const int s = base + threadIdx.x;
-        int w = 0;
-        if (s < p.num_seqs) {
-            const int raw = __ldg(p.context_lens + s);
-            const int L = tc_seq_len(p, s);
-            if (c == 0 && L != raw) flag_error(p.errors, PKV_DEVERR_CONTEXT);
-            w = L > 0 ? (L + 127) / 128 + kTcUnitCost : 0;
+    // a sequence's cost w(s); c == 0 flags lengths out of range
+    auto seq_cost = [&](int s) -> int {
+        if (s >= p.num_seqs) return 0;
+        const int raw = __ldg(p.context_lens + s);
+        const int L = tc_seq_len(p, s);
+        if (c == 0 && L != raw) flag_error(p.errors, PKV_DEVERR_CONTEXT);
+        return L > 0 ? (L + 127) / 128 + kTcUnitCost : 0;
+    };
+    // the CTA whose range holds cost index v0 in sequence s (prefix pre, cost w) notes it
+    auto note_start = [&](int s, int64_t pre, int w, int64_t v0) {
+        if (w > 0 && pre * NU <= v0 && v0 < (pre + w) * NU) {
+            scratch[16] = s;
+            scratch[17] = (int)(v0 - pre * NU);         // offset of the start in s's units
+            scratch[18] = (int)pre;
         }
-        if (base == 0) w_first = w;
-        total += block_sum(w);
-    }
-    const int64_t vtot = total * NU;
-    const int64_t v0 = vtot * c / C, v1 = vtot * (c + 1) / C;
-    if (threadIdx.x == 0) scratch[16] = -1;
-    __syncthreads();
-    {
+    };
+    int64_t v0, v1;
+    if (p.num_seqs <= nthreads) {
+        // one chunk: a single block scan gives every prefix and the total
+        const int s = threadIdx.x;
+        const int w = seq_cost(s);
+        int incl = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(kAll, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) scratch[warp] = incl;
+        if (threadIdx.x == 0) scratch[16] = -1;
+        __syncthreads();
+        int before = 0, all = 0;
+        for (int wp = 0; wp < nwarps; ++wp) {
+            if (wp < warp) before += scratch[wp];
+            all += scratch[wp];
+        }
+        const int64_t vtot = (int64_t)all * NU;
+        v0 = vtot * c / C;
+        v1 = vtot * (c + 1) / C;
+        const int64_t pre = before + incl - w;    // W(s)
+        if (s < p.num_seqs) {
+            if (c == 0) p.prefix[s] = (int32_t)pre;
+            note_start(s, pre, w, v0);
+        }
+        if (c == 0 && threadIdx.x == 0) p.prefix[p.num_seqs] = all;
+    } else {
+        // pass 1: V; pass 2: the prefixes and the sequence holding the start
+        int64_t total = 0;
+        for (int base = 0; base < p.num_seqs; base += nthreads) total += block_sum(seq_cost(base + threadIdx.x));
+        const int64_t vtot = total * NU;
+        v0 = vtot * c / C;
+        v1 = vtot * (c + 1) / C;
+        if (threadIdx.x == 0) scratch[16] = -1;
+        __syncthreads();
         int64_t carry = 0;
         for (int base = 0; base < p.num_seqs; base += nthreads) {
             const int s = base + threadIdx.x;
-            int w = w_first;
-            if (base > 0) w = s < p.num_seqs && tc_seq_len(p, s) > 0 ? (tc_seq_len(p, s) + 127) / 128 + kTcUnitCost : 0;
+            const int w = s < p.num_seqs && tc_seq_len(p, s) > 0 ? (tc_seq_len(p, s) + 127) / 128 + kTcUnitCost : 0;
             int incl = w;                           // inclusive scan over the block
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -290,11 +322,7 @@ __global__ void __launch_bounds__(kDecodeTcThreads, 1)
             const int64_t pre = carry + before + incl - w;    // W(s)
             if (s < p.num_seqs) {
                 if (c == 0) p.prefix[s] = (int32_t)pre;
-                if (w > 0 && pre * NU <= v0 && v0 < (pre + w) * NU) {
-                    scratch[16] = s;
-                    scratch[17] = (int)(v0 - pre * NU);         // offset of the start in s's units
-                    scratch[18] = (int)pre;
-                }
+                note_start(s, pre, w, v0);
             }
             carry += chunk;
             const bool found = __syncthreads_or(scratch[16] >= 0);

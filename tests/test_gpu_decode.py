@@ -118,6 +118,19 @@ def test_groups_beyond_128_heads(dtype, H, D, bs):
     check_step(lay)
 
 
+def test_wide_group_more_sequences_than_threads():
+    """The tensor-core decode's range search scans the lengths one block of
+    threads (352) at a time: 700 sequences take two passes over two chunks,
+    with empty and one-token contexts among them."""
+    rng = np.random.default_rng(71)
+    lens = rng.integers(0, 400, 700)
+    lens[::97] = 0
+    lens[5::89] = 1
+    lay = wl.custom_layout("bf16", num_heads=32, num_kv_heads=2, head_size=128, block_size=16,
+                           context_lens=lens.tolist(), seed=71)
+    check_step(lay)
+
+
 @pytest.mark.parametrize("ps_blocks", [1, 3, 32])
 def test_forced_partitions(ps_blocks):
     lay = wl.custom_layout("bf16", 16, 2, 128, 16, [1, 47, 48, 49, 700, 1025, 2048, 16], seed=3)
