@@ -122,9 +122,14 @@ const char* pkv_version(void);
  *   stream         cudaStream_t (void*), may be NULL
  *
  * Supported: dtype f32/f16/bf16, head_size 64 or 128, block_size 16 or 32,
- * any G, num_seqs <= 16384.  Anything else: PKV_ERR_UNSUPPORTED.  Groups of
- * more than 8 query heads are processed in slices of 8 heads that stream the
- * same K/V tiles at about the same time (the repeats come from L2).
+ * any G, num_seqs <= 16384.  Anything else: PKV_ERR_UNSUPPORTED.  With f16
+ * or bf16 elements, G >= 16 and partition_size 0, the call runs on the
+ * tcgen05 tensor cores: the rows of each product are the group's query heads
+ * (slices of up to 128), and the key tiles of all (sequence, KV head, slice)
+ * units are split into ranges of equal cost over one CTA per SM, whose
+ * partial results the merge kernel combines.  Otherwise groups of more than
+ * 8 query heads are processed in slices of 8 heads that stream the same K/V
+ * tiles at about the same time (the repeats come from L2).
  * ------------------------------------------------------------------------- */
 pkv_status paged_attention_decode(void* out, const void* q, const void* k_cache,
                                   const void* v_cache, const int32_t* block_tables,
