@@ -368,6 +368,12 @@ pkv_status swap_blocks(const void* const* src_caches, void* const* dst_caches, i
  *                  run on the tensor cores with fp32 accumulation and the
  *                  softmax weights rounded to dtype before the product with V
  *
+ * The kernel is persistent (one CTA per SM) and takes its work items from a
+ * counter the library owns: each call takes the next of 64 counters of the
+ * device, and its last CTA leaves it at zero, on every path.  At most 64
+ * prefill calls may run at the same time on one device (streams running in
+ * parallel); calls on one stream run one after another.
+ *
  * Device checks: n < 0, n > L, n > max_query_len, L > max_blocks_per_seq *
  * block_size or queries outside [0, num_tokens) set PKV_DEVERR_CONTEXT and
  * the sequence's rows are not written; a block id outside the pool sets
