@@ -107,9 +107,10 @@ const char* pkv_version(void);
  *                  * block_size (the workspace must then be sized for that)
  *   dtype          element type of q, caches and out (all the same)
  *   partition_size tokens per split-context partition: 0 = library choice
- *                  (a per-call size between 8 and 16 blocks, 16 and 32
- *                  for G >= 4); otherwise a multiple of block_size, at
- *                  most 32 * block_size.  Contexts longer than one partition are
+ *                  (a per-call size between 8 and 16 blocks; for G >= 4,
+ *                  16 and 64, or 16 and 32 over an FP8 cache); otherwise a
+ *                  multiple of block_size, at most 32 * block_size.
+ *                  Contexts longer than one partition are
  *                  processed in parallel pieces whose softmax statistics a
  *                  second kernel merges (log-sum-exp reduction).
  *   workspace      device scratch of at least

@@ -129,7 +129,7 @@ struct Item {
     int ntok;     // tokens in the item (may be 0 for an empty sequence)
     int nblk;     // stages the item occupies (>= 1)
     int whole;    // the item is the whole sequence
-    int tbl;      // lane j holds the item's j-th physical block id
+    int tbl;      // lane j holds the item's (32k + j)-th physical block id (k = issued blocks / 32)
     int64_t slot; // fused cache write: slot of the new token if this item holds it, else -1
 };
 
@@ -818,7 +818,7 @@ using ConsumerFor = typename std::conditional<
 // partition_size], take the largest whose fill ratio (n/NW) / ceil(n/NW) is
 // within 0.02 of the best.
 // ===========================================================================
-constexpr int kMaxPartitionCandidates = 33;
+constexpr int kMaxPartitionCandidates = 49;
 
 __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, const DecodeParams& p,
                                                 int bs) {
@@ -837,15 +837,14 @@ __device__ __forceinline__ int choose_partition(const int* s_len, int nseq, cons
     __syncthreads();
     if (threadIdx.x == 0) {
         const float nw = (float)(gridDim.x * p.warps);
-        float fill[kMaxPartitionCandidates];
-        float best = 0.f;
-        for (int j = 0; j < nc; ++j) {
+        auto fill = [&](int j) {
             const float x = (float)s_count[j] * p.num_kv_heads * p.slices / nw;
-            fill[j] = x / ceilf(x);
-            best = fmaxf(best, fill[j]);
-        }
+            return x / ceilf(x);
+        };
+        float best = 0.f;
+        for (int j = 0; j < nc; ++j) best = fmaxf(best, fill(j));
         int pick = 0;
-        while (fill[pick] < best - 0.02f) ++pick;
+        while (fill(pick) < best - 0.02f) ++pick;
         s_choice = p.partition_size - pick * bs;
     }
     __syncthreads();
@@ -929,6 +928,10 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
     const int n_items = s_pre[nseq] * NV;
     const int NW = gridDim.x * p.warps;
     const int gw = blockIdx.x * p.warps + warp;
+    // Items of more than 32 blocks (partitions up to 64 blocks) only for
+    // 16-bit caches and groups of 4+ heads; elsewhere the host keeps
+    // partitions at 32 blocks or less and this code is left out.
+    constexpr bool kLongItems = !std::is_same<TC, fp8e4m3>::value && G >= 4;
 
     auto fetch = [&](int idx) -> Item {
         Item it;
@@ -980,6 +983,14 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
     auto issue = [&]() {
         if (P.idx >= n_items) return;
         const int st = issue_st;
+        if constexpr (kLongItems) {
+            if (pj > 0 && (pj & 31) == 0) {
+                // the item's next 32 block ids (an item of more than 32 blocks)
+                const int used = (P.ntok + BS - 1) / BS;
+                if (pj + lane < used)
+                    P.tbl = __ldg(p.block_tables + (size_t)P.s * p.max_blocks_per_seq + P.tok0 / BS + pj + lane);
+            }
+        }
         const int phys = __shfl_sync(kFull, P.tbl, pj & 31);
         int nvalid = min(max(P.ntok - pj * BS, 0), BS);
         const bool bad = nvalid > 0 && (phys < 0 || phys >= p.num_blocks);

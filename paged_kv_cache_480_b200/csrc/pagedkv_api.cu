@@ -94,10 +94,12 @@ int resolve_partition(int num_heads, int num_kv_heads, int block_size, int max_c
         if (largest) *largest = requested;
         return requested;
     }
+    // the library's range: [lo, hi] blocks, chosen per call on the device;
+    // lo sizes the workspace (the most partitions)
     const int G = num_heads / num_kv_heads;
-    const int hi = (G >= 4 ? 32 : 16) * block_size;
+    const int lo = (G >= 4 ? 16 : 8) * block_size, hi = (G >= 4 ? 64 : 16) * block_size;
     if (largest) *largest = hi;
-    return hi / 2;
+    return lo;
 }
 
 struct WorkspaceLayout {
@@ -230,6 +232,9 @@ pkv_status decode_impl(void* out, const void* q, const void* k_cache, const void
     const int ps = resolve_partition(num_heads, num_kv_heads, block_size, max_context_len,
                                      partition_size, &ps_hi);
     if (ps == 0) return PKV_ERR_INVALID_ARG;
+    // over an FP8 cache the warps retire blocks twice as fast, so longer
+    // partitions leave too few items per warp: at most 32 blocks there
+    if (fp8_cache && ps_hi > 32 * block_size) ps_hi = 32 * block_size;
     const bool tc = !fp8_cache && app == nullptr && use_decode_tc(num_heads, num_kv_heads, dtype, partition_size);
     const WorkspaceLayout wl =
         workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, ps, tc);
