@@ -263,7 +263,7 @@ struct FmaConsumer {
 #pragma unroll
             for (int d = 0; d < DL; ++d) acc[d] += __shfl_xor_sync(kFull, acc[d], off);
         }
-        if (u != 0 || h >= mt.nh) return;
+        if (u != 0 || h >= (G <= 2 ? G : mt.nh)) return;
         if (mt.flags & kWhole) {
             const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
             uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<TQ*>(p.out) + (size_t)(mt.obase + h) * D);
@@ -478,7 +478,7 @@ struct MmaConsumer {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int head = 2 * c + e;
-            if (head >= mt.nh) continue;
+            if (head >= (G <= 2 ? G : mt.nh)) continue;
             const float lt = e ? t1 : t0;
             if (mt.flags & kWhole) {
                 const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
@@ -764,7 +764,7 @@ struct MmaConsumerFp8 {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int head = 2 * c + e;
-            if (head >= mt.nh) continue;
+            if (head >= (G <= 2 ? G : mt.nh)) continue;
             const float lt = e ? t1 : t0;
             if (mt.flags & kWhole) {
                 const float inv = lt > 0.f ? p.v_scale / lt : 0.f;
@@ -1090,7 +1090,8 @@ __global__ void __launch_bounds__(decode_max_threads<TQ, TC, G>(), 1) paged_deco
         } else {
             mt = meta[cons_st];
         }
-        if (mt.flags & kFirst) cons.begin(qbuf + meta[cons_st].qslot * S::QBYTES, qscale, meta[cons_st].nh);
+        // (a column count of 1 or 2 only ever holds a whole group of that size)
+        if (mt.flags & kFirst) cons.begin(qbuf + meta[cons_st].qslot * S::QBYTES, qscale, G <= 2 ? G : meta[cons_st].nh);
         using Cons = ConsumerFor<TQ, TC, D, BS, G>;
         if constexpr (Cons::kPairs) {
             // the item's next block is in the next stage: take both together
